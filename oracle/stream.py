@@ -1,0 +1,120 @@
+"""A stream of frames through rotate -> append -> attend -> commit/rollback, float64.
+
+TEST INFRASTRUCTURE ONLY (see ``oracle/__init__``).
+
+Per frame ([3DRoPE-KV] "Frame Appending and Position Encoding Integration" and
+"Attention Computation with Cached RoPE"; [KVBenefits] "Dynamic Keyframe Selection"):
+
+1. rotate the frame's q and k at their 3D positions (``rope3d``), v unrotated;
+2. append: the patch keys/values take a page popped from the free list, the 6 special
+   tokens take the next slots of the special stream (``retention``);
+3. attend: the frame's queries over scale pages -> window pages -> own page -> specials
+   (``attention.attend``);
+4. commit (keyframe: deferred eviction) or roll back (non-keyframe).
+
+Only the K/V of frames still retained are kept, so long streams stay bounded in memory,
+unless ``keep_history`` is set (small streams; enables the masked whole-history check).
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+
+from . import attention, retention, rope3d
+
+
+@dataclass
+class FrameResult:
+    frame_idx: int
+    is_keyframe: bool
+    page: int
+    special_slot: int
+    visible: retention.Visible
+    visible_frames: list       # frames whose patch pages are visible, visible order
+    q_rot: np.ndarray          # [T, H, D] fp64
+    k_rot: np.ndarray          # [T, H, D] fp64
+    rows: np.ndarray           # query rows computed
+    out: np.ndarray            # [len(rows), H, D] fp64
+    lse: np.ndarray            # [len(rows), H] natural-log sum-exp of scaled scores
+    evicted: int | None
+    state: dict                # retention snapshot after commit / rollback
+
+
+class StreamOracle:
+    def __init__(self, heads: int, head_dim: int, pph: int, ppw: int, scale_frames: int,
+                 sliding_window: int, max_frames: int, specials_per_frame: int = 6,
+                 theta: float = rope3d.THETA, keep_history: bool = False):
+        self.heads = heads
+        self.head_dim = head_dim
+        self.pph = pph
+        self.ppw = ppw
+        self.psi = specials_per_frame
+        self.theta = theta
+        self.ret = retention.PagedRetention(scale_frames, sliding_window, max_frames,
+                                            specials_per_frame)
+        self.patch_kv: dict = {}      # frame -> (k [Pf,H,D], v [Pf,H,D]) of retained frames
+        self.special_kv: list = []    # [(frame, k [6,H,D], v [6,H,D])] committed, in order
+        self.keep_history = keep_history
+        self.history: list = []       # [(frame, k [T,H,D], v [T,H,D])] every frame seen
+
+    @property
+    def tokens_per_frame(self) -> int:
+        return self.psi + self.pph * self.ppw
+
+    def reset(self) -> None:
+        self.ret.reset()
+        self.patch_kv = {}
+        self.special_kv = []
+        self.history = []
+
+    def step(self, frame_idx: int, is_keyframe: bool, q: np.ndarray, k: np.ndarray,
+             v: np.ndarray, rows=None) -> FrameResult:
+        T = self.tokens_per_frame
+        assert q.shape == (T, self.heads, self.head_dim), q.shape
+        page, slot = self.ret.append(frame_idx, is_keyframe)
+        qr = rope3d.rotate_frame(q, frame_idx, self.psi, self.pph, self.ppw, self.theta)
+        kr = rope3d.rotate_frame(k, frame_idx, self.psi, self.pph, self.ppw, self.theta)
+        v64 = np.asarray(v, dtype=np.float64)
+        vis = self.ret.visible()
+
+        frames = self.ret.retained_frames()
+        ks = [self.patch_kv[f][0] for f in frames] + [kr[self.psi:]]
+        vs = [self.patch_kv[f][1] for f in frames] + [v64[self.psi:]]
+        ks += [e[1] for e in self.special_kv] + [kr[:self.psi]]
+        vs += [e[2] for e in self.special_kv] + [v64[:self.psi]]
+        K = np.concatenate(ks, axis=0)
+        V = np.concatenate(vs, axis=0)
+        assert K.shape[0] == len(vis.patch_pages) * self.pph * self.ppw + vis.n_special
+
+        rows = np.arange(T) if rows is None else np.asarray(rows)
+        out, lse = attention.attend(qr[rows], K, V, return_lse=True)
+
+        if self.keep_history:
+            self.history.append((frame_idx, kr, v64))
+        evicted_frame = None
+        if is_keyframe and len(self.ret.scale) >= self.ret.scale_frames \
+                and len(self.ret.window) >= self.ret.sliding_window:
+            evicted_frame = self.ret.window[0][1] if self.ret.sliding_window > 0 else frame_idx
+        evicted = self.ret.finish()
+        if is_keyframe:
+            self.patch_kv[frame_idx] = (kr[self.psi:], v64[self.psi:])
+            self.special_kv.append((frame_idx, kr[:self.psi], v64[:self.psi]))
+            if evicted is not None:
+                del self.patch_kv[evicted_frame]
+        return FrameResult(frame_idx, is_keyframe, page, slot, vis, frames + [frame_idx],
+                           qr, kr, rows, out, lse, evicted, self.ret.snapshot())
+
+    def attend_history_masked(self, q_rot: np.ndarray, frame_idx: int,
+                              committed_before: list) -> np.ndarray:
+        """Whole-history masked attention for the frame just stepped (keep_history only)."""
+        assert self.keep_history
+        frames = [h[0] for h in self.history]
+        K = np.concatenate([h[1] for h in self.history], axis=0)
+        V = np.concatenate([h[2] for h in self.history], axis=0)
+        retained = retention.retained_closed_form(committed_before, self.ret.scale_frames,
+                                                  self.ret.sliding_window)
+        mask = attention.history_mask(frames, frame_idx, committed_before, retained,
+                                      self.psi, self.tokens_per_frame)
+        return attention.attend_masked(q_rot, K, V, mask)
