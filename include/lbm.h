@@ -1,0 +1,220 @@
+/*
+ * lbm.h - C ABI of the streaming-frame step: 3D RoPE, dual-stream paged KV cache, paged
+ * attention, for one NVIDIA B200 (sm_100a).
+ *
+ * The operations follow five articles about the lingbot-map project, cited by title and
+ * section:
+ *   [3DRoPE-KV]  "How 3D RoPE Positional Encoding Works with the Paged KV Cache in
+ *                 LingBot-Map"
+ *   [VideoRoPE]  "Video RoPE Positional Encoding: 3D Rotary Embeddings for Long-Sequence
+ *                 Video in Ling-Bot-Map"
+ *   [RealTime3D] "How LingBot-Map Achieves Real-Time 3D Reconstruction: Streaming
+ *                 Transformers and KV Caching"
+ *   [KVBenefits] "KV Caching Benefits in Ling Bot-Map: 7 Advantages for Streaming Vision
+ *                 Models"
+ *
+ * Conventions common to every call
+ * --------------------------------
+ *  - Every call returns an lbm status (LBM_OK == 0, errors < 0).  Nothing throws or aborts
+ *    across the ABI.  A call that fails leaves the library state as it was.
+ *  - q, k, v and out are DEVICE pointers owned by the caller, contiguous [T][heads][head_dim]
+ *    (token-major), T = specials_per_frame + patches_per_frame, 16-byte aligned, element type
+ *    the cache's dtype (LBM_F32: float, LBM_BF16: bfloat16).
+ *  - stream is a cudaStream_t (NULL = the legacy default stream).  Work is only enqueued;
+ *    nothing synchronises the host except the calls that say so.  Calls on one cache from
+ *    several streams are ordered by the library through an event it records after each launch.
+ *  - The library owns the RoPE tables, the K/V page pools, split-KV scratch and the page
+ *    table.  The caller owns its q/k/v/out buffers and the streams.
+ *  - Host bookkeeping (page table, free list, deferred eviction) runs at call time on the
+ *    host; the only host->device traffic of a frame is kernel launch parameters.
+ */
+#ifndef LBM_H
+#define LBM_H
+
+#if defined(__GNUC__)
+#define LBM_API __attribute__((visibility("default")))
+#else
+#define LBM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ---------------------------------------------------------------------- */
+enum {
+  LBM_OK = 0,
+  LBM_ERR_INVALID = -1,      /* bad argument: null/misaligned pointer, size out of range    */
+  LBM_ERR_UNSUPPORTED = -2,  /* valid but not implemented (head_dim not 64/128, dtype)        */
+  LBM_ERR_SEQUENCE = -3,     /* call out of order (append twice, attend first, frame order)  */
+  LBM_ERR_CAPACITY = -4,     /* special stream full: max_frames keyframes already committed  */
+  LBM_ERR_NOMEM = -5,        /* device or host allocation failed                             */
+  LBM_ERR_CUDA = -6,         /* a CUDA runtime / driver call or kernel launch failed         */
+  LBM_ERR_TIMEOUT = -7       /* a kernel gave up a bounded wait and flagged an error         */
+};
+
+enum { LBM_F32 = 0, LBM_BF16 = 1 };
+
+/* which pool lbm_cache_read_kv copies */
+enum { LBM_K_PATCH = 0, LBM_V_PATCH = 1, LBM_K_SPECIAL = 2, LBM_V_SPECIAL = 3 };
+
+/* Tokens per page of the special stream.  [3DRoPE-KV] "Attention Computation with Cached
+ * RoPE" passes the valid length of the last, partly filled special page; the pages give no
+ * page size, this library uses the attention tile height. */
+#define LBM_SPECIAL_PAGE 128
+/* Most patch pages one frame can see (scale_frames + sliding_window + 1). */
+#define LBM_MAX_PAGES 1024
+
+typedef struct lbm_rope lbm_rope_t;
+typedef struct lbm_cache lbm_cache_t;
+typedef struct lbm_pager lbm_pager_t;
+
+/* ---- 3D RoPE tables ---------------------------------------------------------------------
+ * [3DRoPE-KV] "Multi-Axis Frequency Generation"; [VideoRoPE] "The Three Rotary Dimensions".
+ * One 1D table per axis a in (t, h, w): angle(p, i) = p * theta^(-2i/d_a), i < d_a/2, with
+ * d_h = d_w = 2*(head_dim/6) and d_t = head_dim - 2*d_h; pairs ordered t, h, w along
+ * head_dim/2.  Angles and cos/sin are computed in double on the host and rounded once to
+ * float.  Rows: t in [0, ppf), h in [0, pph], w in [0, ppw].  Token j of frame t sits at
+ * (t, 0, 0) for j < patch_start_idx (special tokens) and at (t, 1 + r, 1 + c) for patch
+ * (r, c) = divmod(j - patch_start_idx, ppw).  Feature pair i is (x[2i], x[2i+1]).
+ *   head_dim       64 or 128 (any even value >= 6 is accepted here; caches take 64/128)
+ *   ppf            frames covered by the t table (frame_idx must stay below it)
+ *   pph, ppw       patch grid of a frame
+ *   patch_start_idx special tokens before the patches of each frame (6)
+ *   theta          base (10000.0); NTK scaling is theta * ntk_factor, passed pre-multiplied
+ *   out            receives the table object; the caller frees it with lbm_rope_destroy
+ *                  after every cache that uses it is destroyed.
+ * Allocates device memory on the current device; synchronous. */
+LBM_API int lbm_rope3d_tables(int head_dim, int ppf, int pph, int ppw, int patch_start_idx,
+                      double theta, lbm_rope_t** out);
+
+/* Writes the expanded table of [3DRoPE-KV] "Multi-Axis Frequency Generation": cos and sin,
+ * each float [ppf * (patch_start_idx + pph*ppw)][head_dim/2] (device pointers, caller-owned),
+ * frames 0..ppf-1 in order, tokens of a frame in the order above.  Enqueued on stream. */
+LBM_API int lbm_rope3d_expand(const lbm_rope_t* rope, float* cos_out, float* sin_out, void* stream);
+
+LBM_API void lbm_rope_destroy(lbm_rope_t* rope);
+
+/* ---- the dual-stream paged KV cache -----------------------------------------------------
+ * [3DRoPE-KV] "Dual-Stream Memory Layout": the patch stream keeps one page of
+ * patches_per_frame tokens per frame; the first scale_frames keyframes' pages stay, the next
+ * sliding_window pages are recycled, the oldest window page returns to a free list when the
+ * window overflows (after the attention of the frame that overflows it: deferred eviction).
+ * The special stream is append-only, specials_per_frame tokens per committed keyframe.
+ *   heads, head_dim    head_dim 64 or 128 (else LBM_ERR_UNSUPPORTED)
+ *   patches_per_frame  must equal rope's pph*ppw
+ *   specials_per_frame must equal rope's patch_start_idx and be 6
+ *   scale_frames, sliding_window  >= 0; scale_frames + sliding_window + 1 <= LBM_MAX_PAGES
+ *   max_frames         keyframes the special stream can hold (>= 1)
+ *   dtype              LBM_BF16 (tensor-core path) or LBM_F32 (exact SIMT path)
+ *   rope               tables built for the same head_dim / grid; must outlive the cache
+ * Device memory: K and V patch pools [heads][P*stride][head_dim] with P = scale_frames +
+ * sliding_window + 1 pages and stride = patches_per_frame rounded up to 128 (zero-filled);
+ * K and V special pools [heads][cap][head_dim], cap = 6*(max_frames+1) rounded up to 128;
+ * split-KV scratch.  Synchronous. */
+LBM_API int lbm_cache_create(int heads, int head_dim, int patches_per_frame, int specials_per_frame,
+                     int scale_frames, int sliding_window, int max_frames, int dtype,
+                     const lbm_rope_t* rope, lbm_cache_t** out);
+
+/* Rotate and append one frame.  [3DRoPE-KV] "Frame Appending and Position Encoding
+ * Integration" and "Complex-Valued Tensor Application"; [VideoRoPE] "Temporal Consistency
+ * in KV-Cache Streaming" (t = absolute frame index).
+ *   q      device, [T][heads][head_dim]; rotated IN PLACE (read, rotated, written back)
+ *   k, v   device, [T][heads][head_dim]; k is rotated, v is not; both are written into the
+ *          frame's patch page (tokens >= 6) and the next 6 slots of the special stream
+ *   frame_idx    strictly greater than the previous frame's, and < rope's ppf
+ *   is_keyframe  1: the frame is kept after its attention; 0: rolled back after it
+ *                ([KVBenefits] "Reduced KV Growth via Keyframe Streaming")
+ * One kernel launch.  Errors: LBM_ERR_SEQUENCE if a frame is already pending or frame_idx
+ * does not increase or is >= ppf; LBM_ERR_CAPACITY for a keyframe when max_frames keyframes
+ * are committed. */
+LBM_API int lbm_append_frame(lbm_cache_t* cache, void* q, const void* k, const void* v,
+                     long long frame_idx, int is_keyframe, void* stream);
+
+/* Attention of the pending frame's (already rotated) queries over what the cache retains:
+ * scale pages -> window pages (oldest first) -> the frame's own page -> all special tokens
+ * ([3DRoPE-KV] "Attention Computation with Cached RoPE"); a frame's own tokens all see each
+ * other; softmax scale 1/sqrt(head_dim).  Then commits the frame (keyframe; deferred
+ * eviction) or rolls it back ([KVBenefits] "Dynamic Keyframe Selection").
+ *   q    device [T][heads][head_dim], the q rotated by lbm_append_frame
+ *   out  device [T][heads][head_dim], written
+ * bf16: one tcgen05 kernel launch, plus one combine launch when the keys are split across
+ * CTAs.  Errors: LBM_ERR_SEQUENCE if no frame is pending. */
+LBM_API int lbm_attend_frame(lbm_cache_t* cache, const void* q, void* out, void* stream);
+
+/* Forget every frame: all pages free, special stream empty ([KVBenefits] "Cross-Window
+ * Alignment for Long Videos": clean_kv_cache).  Host-only; pool contents are left as they
+ * are (nothing reads them before they are written again). */
+LBM_API int lbm_cache_reset(lbm_cache_t* cache);
+
+/* Host snapshot of the page table, for tests and monitoring ([KVBenefits] "Working with
+ * the KV Cache API": get_kv_cache_info).  The caller sets capacity and the five array
+ * pointers (each with room for capacity entries, or NULL to skip); counts are always set. */
+typedef struct {
+  int num_pages;          /* P = scale_frames + sliding_window + 1                          */
+  int n_scale;            /* scale pages held                                                */
+  int n_window;           /* window pages held                                               */
+  int n_free;             /* pages on the free stack                                         */
+  int n_special;          /* committed special tokens                                        */
+  int special_pages;      /* ceil(n_special / LBM_SPECIAL_PAGE)                              */
+  int last_page_len;      /* valid tokens in the last committed special page (0 if none)    */
+  int pending;            /* 1 between lbm_append_frame and lbm_attend_frame                 */
+  int pending_page;       /* page of the pending frame (-1 if none)                         */
+  int pending_is_keyframe;
+  long long pending_frame;
+  long long last_frame;   /* last appended frame_idx, -1 if none                             */
+  long long device_bytes; /* pool + scratch bytes held on the device                         */
+  long long kernel_launches; /* kernels this cache has launched since it was created         */
+  int capacity;           /* in: entries each array below can take                           */
+  int* scale_pages;       /* out: scale pages in commit order                                */
+  long long* scale_frames;
+  int* window_pages;      /* out: window pages oldest first                                  */
+  long long* window_frames;
+  int* free_pages;        /* out: free stack bottom .. top (top is popped next)              */
+} lbm_cache_state_t;
+
+LBM_API int lbm_cache_state(const lbm_cache_t* cache, lbm_cache_state_t* state);
+
+/* Copies part of a pool to host memory (synchronises the device; for tests).
+ *   which  LBM_K_PATCH / LBM_V_PATCH: index = page id, count ignored; host_out receives
+ *          [heads][patches_per_frame][head_dim]
+ *          LBM_K_SPECIAL / LBM_V_SPECIAL: tokens [index, index+count) of the special
+ *          stream; host_out receives [heads][count][head_dim]
+ * Elements are the cache's dtype. */
+LBM_API int lbm_cache_read_kv(const lbm_cache_t* cache, int which, int index, int count,
+                      void* host_out);
+
+/* Synchronises the device and reports a bounded wait that ran out in an earlier kernel
+ * (LBM_ERR_TIMEOUT, after which the error word is cleared) or LBM_OK. */
+LBM_API int lbm_cache_check(lbm_cache_t* cache);
+
+LBM_API void lbm_cache_destroy(lbm_cache_t* cache);
+
+LBM_API const char* lbm_status_string(int status);
+
+/* ---- host-only page manager -------------------------------------------------------------
+ * The page table / free list / deferred-eviction state machine the cache drives, exposed on
+ * its own so that it can be checked without a GPU.  Same rules as the cache:
+ * [3DRoPE-KV] "Dual-Stream Memory Layout"; [KVBenefits] "Dynamic Keyframe Selection".
+ * A fresh manager pops pages 0, 1, ..., P-1; evicted and rolled-back pages are pushed on
+ * top of the free stack (LIFO). */
+LBM_API int lbm_pager_create(int scale_frames, int sliding_window, int max_frames,
+                     int specials_per_frame, lbm_pager_t** out);
+/* Pops the frame's page and reserves its special slots; *page and *special_slot receive them. */
+LBM_API int lbm_pager_append(lbm_pager_t* pager, long long frame_idx, int is_keyframe, int* page,
+                     int* special_slot);
+/* The pending frame's visible patch pages (scale, window oldest first, own page) into
+ * pages[0..capacity), their count, and the visible special tokens (committed + own). */
+LBM_API int lbm_pager_visible(const lbm_pager_t* pager, int* pages, int capacity, int* n_pages,
+                      int* n_special, int* last_page_len);
+/* Commit (keyframe) or roll back (non-keyframe) the pending frame; *evicted receives the
+ * page returned to the free list by deferred eviction, or -1. */
+LBM_API int lbm_pager_finish(lbm_pager_t* pager, int* evicted);
+LBM_API int lbm_pager_reset(lbm_pager_t* pager);
+LBM_API int lbm_pager_state(const lbm_pager_t* pager, lbm_cache_state_t* state);
+LBM_API void lbm_pager_destroy(lbm_pager_t* pager);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LBM_H */

@@ -33,11 +33,11 @@ def attend(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float | None = No
     v = np.asarray(v, dtype=np.float64)
     if scale is None:
         scale = 1.0 / np.sqrt(q.shape[-1])
-    s = np.einsum("thd,nhd->htn", q, k) * scale          # [H, T, N]
+    s = np.matmul(q.transpose(1, 0, 2), k.transpose(1, 2, 0)) * scale   # [H, T, N]
     m = s.max(axis=-1, keepdims=True)
     p = np.exp(s - m)
     l = p.sum(axis=-1, keepdims=True)
-    out = np.einsum("htn,nhd->thd", p / l, v)
+    out = np.matmul(p / l, v.transpose(1, 0, 2)).transpose(1, 0, 2)      # [T, H, D]
     if return_lse:
         return out, (m[..., 0] + np.log(l[..., 0])).T
     return out
@@ -51,12 +51,12 @@ def attend_masked(q: np.ndarray, k: np.ndarray, v: np.ndarray, mask: np.ndarray,
     v = np.asarray(v, dtype=np.float64)
     if scale is None:
         scale = 1.0 / np.sqrt(q.shape[-1])
-    s = np.einsum("thd,nhd->htn", q, k) * scale
+    s = np.matmul(q.transpose(1, 0, 2), k.transpose(1, 2, 0)) * scale
     s = np.where(np.asarray(mask, dtype=bool)[None, None, :], s, -np.inf)
     m = s.max(axis=-1, keepdims=True)
     p = np.exp(s - m)
     p = p / p.sum(axis=-1, keepdims=True)
-    return np.einsum("htn,nhd->thd", p, v)
+    return np.matmul(p, v.transpose(1, 0, 2)).transpose(1, 0, 2)
 
 
 def history_mask(frames: list, current: int, committed_before: list, retained_before: list,

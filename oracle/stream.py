@@ -24,6 +24,8 @@ import numpy as np
 
 from . import attention, retention, rope3d
 
+ROW_CHUNK = 64
+
 
 @dataclass
 class FrameResult:
@@ -45,7 +47,11 @@ class FrameResult:
 class StreamOracle:
     def __init__(self, heads: int, head_dim: int, pph: int, ppw: int, scale_frames: int,
                  sliding_window: int, max_frames: int, specials_per_frame: int = 6,
-                 theta: float = rope3d.THETA, keep_history: bool = False):
+                 theta: float = rope3d.THETA, keep_history: bool = False, kv_source=None):
+        """kv_source, if given, is a callable (frame, region) -> (k, v) returning a past
+        frame's unrotated inputs (region "patch": [pph*ppw, H, D], "special": [6, H, D]);
+        the oracle then keeps no K/V of its own and re-creates retained keys when a frame
+        attends, which keeps long streams small in memory."""
         self.heads = heads
         self.head_dim = head_dim
         self.pph = pph
@@ -58,6 +64,7 @@ class StreamOracle:
         self.special_kv: list = []    # [(frame, k [6,H,D], v [6,H,D])] committed, in order
         self.keep_history = keep_history
         self.history: list = []       # [(frame, k [T,H,D], v [T,H,D])] every frame seen
+        self.kv_source = kv_source
 
     @property
     def tokens_per_frame(self) -> int:
@@ -69,8 +76,23 @@ class StreamOracle:
         self.special_kv = []
         self.history = []
 
+    def _retained_kv(self, frame: int, region: str):
+        """Rotated k and plain v of a retained frame's patches or specials (fp64)."""
+        if self.kv_source is None:
+            if region == "patch":
+                return self.patch_kv[frame]
+            for f, ks, vs in self.special_kv:
+                if f == frame:
+                    return ks, vs
+            raise KeyError(frame)
+        k, v = self.kv_source(frame, region)
+        pos = rope3d.token_positions(frame, self.psi, self.pph, self.ppw)
+        pos = pos[self.psi:] if region == "patch" else pos[:self.psi]
+        kr = rope3d.rotate(k, rope3d.angles_for_positions(pos, self.head_dim, self.theta))
+        return kr, np.asarray(v, dtype=np.float64)
+
     def step(self, frame_idx: int, is_keyframe: bool, q: np.ndarray, k: np.ndarray,
-             v: np.ndarray, rows=None) -> FrameResult:
+             v: np.ndarray, rows=None, attend: bool = True) -> FrameResult:
         T = self.tokens_per_frame
         assert q.shape == (T, self.heads, self.head_dim), q.shape
         page, slot = self.ret.append(frame_idx, is_keyframe)
@@ -80,16 +102,36 @@ class StreamOracle:
         vis = self.ret.visible()
 
         frames = self.ret.retained_frames()
-        ks = [self.patch_kv[f][0] for f in frames] + [kr[self.psi:]]
-        vs = [self.patch_kv[f][1] for f in frames] + [v64[self.psi:]]
-        ks += [e[1] for e in self.special_kv] + [kr[:self.psi]]
-        vs += [e[2] for e in self.special_kv] + [v64[:self.psi]]
-        K = np.concatenate(ks, axis=0)
-        V = np.concatenate(vs, axis=0)
-        assert K.shape[0] == len(vis.patch_pages) * self.pph * self.ppw + vis.n_special
-
         rows = np.arange(T) if rows is None else np.asarray(rows)
-        out, lse = attention.attend(qr[rows], K, V, return_lse=True)
+        if attend and len(rows):
+            ks, vs = [], []
+            for f in frames:
+                kf, vf = self._retained_kv(f, "patch")
+                ks.append(kf)
+                vs.append(vf)
+            ks.append(kr[self.psi:])
+            vs.append(v64[self.psi:])
+            for f in self.committed_frames():
+                kf, vf = self._retained_kv(f, "special")
+                ks.append(kf)
+                vs.append(vf)
+            ks.append(kr[:self.psi])
+            vs.append(v64[:self.psi])
+            K = np.concatenate(ks, axis=0)
+            V = np.concatenate(vs, axis=0)
+            assert K.shape[0] == len(vis.patch_pages) * self.pph * self.ppw + vis.n_special
+            # rows are independent, so the query rows are taken in chunks to bound memory
+            outs, lses = [], []
+            for c in range(0, len(rows), ROW_CHUNK):
+                o, e = attention.attend(qr[rows[c:c + ROW_CHUNK]], K, V, return_lse=True)
+                outs.append(o)
+                lses.append(e)
+            out = np.concatenate(outs, axis=0)
+            lse = np.concatenate(lses, axis=0)
+        else:
+            rows = rows[:0]
+            out = np.zeros((0, self.heads, self.head_dim))
+            lse = np.zeros((0, self.heads))
 
         if self.keep_history:
             self.history.append((frame_idx, kr, v64))
@@ -98,13 +140,17 @@ class StreamOracle:
                 and len(self.ret.window) >= self.ret.sliding_window:
             evicted_frame = self.ret.window[0][1] if self.ret.sliding_window > 0 else frame_idx
         evicted = self.ret.finish()
-        if is_keyframe:
+        if is_keyframe and self.kv_source is None:
             self.patch_kv[frame_idx] = (kr[self.psi:], v64[self.psi:])
             self.special_kv.append((frame_idx, kr[:self.psi], v64[:self.psi]))
             if evicted is not None:
                 del self.patch_kv[evicted_frame]
         return FrameResult(frame_idx, is_keyframe, page, slot, vis, frames + [frame_idx],
                            qr, kr, rows, out, lse, evicted, self.ret.snapshot())
+
+    def committed_frames(self) -> list:
+        """Committed keyframes in commit order (their specials are all visible)."""
+        return list(self.ret.committed)
 
     def attend_history_masked(self, q_rot: np.ndarray, frame_idx: int,
                               committed_before: list) -> np.ndarray:

@@ -1,0 +1,629 @@
+// Paged attention of one frame's queries over the retained keys, bf16 in / fp32 softmax,
+// on the 5th-generation tensor cores (tcgen05, accumulators in tensor memory).
+//
+// [3DRoPE-KV] "Attention Computation with Cached RoPE": the queries of the frame attend
+// over the visible page table (scale pages -> window pages -> own page -> special pages,
+// the last special page partly filled), with K/V that already carry their rotation.
+//
+// One CTA = one (query tile of 128 rows, split of the key tiles, head).  Warp roles:
+//   warp 0      TMA producer: Q tile once, then K/V tiles gathered page by page through
+//               the page table into a ring of shared-memory stages (128B swizzle).
+//   warp 1      allocates tensor memory; one lane issues every tcgen05.mma:
+//                 S_j = Q K_j^T   (A, B from shared memory)      -> TMEM S[j%2]
+//                 O  += P_j V_j   (A = P from TMEM, B = V smem)   -> TMEM O
+//               S_{j+1} is issued before waiting for P_j, so the tensor core works on the
+//               next scores while the softmax warps work on this tile.
+//   warps 2..5  softmax: each thread owns one query row (its TMEM lane); reads S_j,
+//               row max, exp2, row sum in fp32, writes P_j (bf16) into TMEM, and
+//               rescales O only when the running max grew by more than 2^8 (lazy
+//               rescale; exact because O and l always share the same reference max).
+// Tensor memory (512 columns): S0 [0,128) S1 [128,256) P0 [256,320) P1 [320,384)
+// O [384, 384+D).
+// Every mbarrier wait is bounded (about 2 s); a wait that runs out sets the device error
+// word, raises a CTA-wide abort flag, and every role falls through to the common exit,
+// which drains outstanding copies / MMAs (bounded) and frees tensor memory.
+#include <cuda_bf16.h>
+
+#include "../../include/lbm.h"
+#include "lbm_internal.h"
+
+namespace lbm {
+namespace {
+
+constexpr int BM = 128;         // query rows per CTA
+constexpr int BN = 128;         // keys per tile
+constexpr int kThreads = 192;   // 6 warps
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t TM_S = 0;    // S buffer b at TM_S + 128 b
+constexpr uint32_t TM_P = 256;  // P buffer b at TM_P + 64 b
+constexpr uint32_t TM_O = 384;
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when max grows by > 2^8
+constexpr unsigned kFull = 0xffffffffu;
+
+template <int D>
+struct Cfg {
+  static constexpr int NS = D == 64 ? 4 : 3;            // K/V pipeline stages
+  static constexpr int ATOM_BYTES = 128 * 128;          // 128 rows x 64 bf16 (one swizzle atom column)
+  static constexpr int ATOMS = D / 64;
+  static constexpr int TILE_BYTES = ATOMS * ATOM_BYTES; // one Q, K or V tile
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + TILE_BYTES;
+  static constexpr int OFF_V = OFF_K + NS * TILE_BYTES;
+  static constexpr int OFF_BAR = OFF_V + NS * TILE_BYTES;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM = OFF_BAR + BAR_BYTES + 1024;  // + slack to align the base to 1 KB
+};
+
+// ---- PTX wrappers -----------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ unsigned long long global_timer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait for the phase of `bar` with the given parity to complete.  Returns false
+// when the CTA is aborting or the limit ran out (then the error word and abort flag are set).
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                       int* err, int where) {
+  if (mbar_try(bar, parity)) return true;
+  const unsigned long long t0 = global_timer();
+  while (true) {
+    if (mbar_try(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (global_timer() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      atomicExch(err, where);
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* tm, int x, int y,
+                                            int z, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor (sm100 format, version 1, 128-byte swizzle).
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor of kind::f16: bf16 x bf16 -> f32, K-major A, B K- or MN-major.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accum)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accum)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+      : "memory");
+}
+
+// 32 consecutive 32-bit columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Pins registers after tcgen05.wait::ld so no use is scheduled before the wait.
+template <int N>
+__device__ __forceinline__ void reg_fence(uint32_t* r) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i])::"memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+      "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]),
+      "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&b);
+}
+
+// Key tile t of the visible list: pool (patch or special), first pool row, valid keys.
+struct TileRef {
+  bool special;
+  int row0;
+  int valid;
+};
+
+__device__ __forceinline__ TileRef tile_ref(const AttnParams& p, int t) {
+  const int npt = p.n_pages * p.tiles_per_page;
+  TileRef r;
+  if (t < npt) {
+    const int pi = t / p.tiles_per_page;
+    const int i = t - pi * p.tiles_per_page;
+    r.special = false;
+    r.row0 = (int)p.pages[pi] * p.page_stride + BN * i;
+    r.valid = min(BN, p.patches - BN * i);
+  } else {
+    const int i = t - npt;
+    r.special = true;
+    r.row0 = BN * i;
+    r.valid = min(BN, p.n_special - BN * i);
+  }
+  return r;
+}
+
+struct Bars {
+  uint64_t q_full;
+  uint64_t s_full[2];
+  uint64_t s_free[2];
+  uint64_t p_full[2];
+  uint64_t pv_done[2];
+  uint64_t drain;
+  uint64_t kv_full[4];
+  uint64_t kv_empty[4];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_tc_kernel(const __grid_constant__ AttnParams p) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  Bars* bars = reinterpret_cast<Bars*>(smem + C::OFF_BAR);
+  volatile int* abort_flag = &bars->abort_flag;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int q_tile = blockIdx.x;
+  const int split = blockIdx.y;
+  const int head = blockIdx.z;
+  const int t_begin = split * p.tiles_per_split;
+  const int t_end = min(p.n_tiles, t_begin + p.tiles_per_split);
+  const int n = t_end - t_begin;
+
+  const uint32_t sQ = smem_u32(smem + C::OFF_Q);
+  const uint32_t sK = smem_u32(smem + C::OFF_K);
+  const uint32_t sV = smem_u32(smem + C::OFF_V);
+  auto bar = [&](const uint64_t& b) { return smem_u32(&b); };
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(bars->q_full), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(bars->s_full[b]), 1);
+      mbar_init(bar(bars->s_free[b]), 128);
+      mbar_init(bar(bars->p_full[b]), 128);
+      mbar_init(bar(bars->pv_done[b]), 1);
+    }
+    mbar_init(bar(bars->drain), 1);
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(bar(bars->kv_full[s]), 1);
+      mbar_init(bar(bars->kv_empty[s]), 1);
+    }
+    bars->abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&bars->tmem_base)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int issued = 0;
+      mbar_expect_tx(bar(bars->q_full), C::TILE_BYTES);
+#pragma unroll
+      for (int a = 0; a < C::ATOMS; ++a)
+        tma_load_3d(sQ + a * C::ATOM_BYTES, &p.tm_q, 64 * a, head, q_tile * BM,
+                    bar(bars->q_full));
+      for (int j = 0; j < n; ++j) {
+        const int s = j % C::NS;
+        if (j >= C::NS &&
+            !mbar_wait(bar(bars->kv_empty[s]), ((j - C::NS) / C::NS) & 1, abort_flag, p.err, 1))
+          break;
+        const TileRef t = tile_ref(p, t_begin + j);
+        const CUtensorMap* tk = t.special ? &p.tm_ks : &p.tm_kp;
+        const CUtensorMap* tv = t.special ? &p.tm_vs : &p.tm_vp;
+        mbar_expect_tx(bar(bars->kv_full[s]), 2 * C::TILE_BYTES);
+#pragma unroll
+        for (int a = 0; a < C::ATOMS; ++a) {
+          tma_load_3d(sK + s * C::TILE_BYTES + a * C::ATOM_BYTES, tk, 64 * a, t.row0, head,
+                      bar(bars->kv_full[s]));
+          tma_load_3d(sV + s * C::TILE_BYTES + a * C::ATOM_BYTES, tv, 64 * a, t.row0, head,
+                      bar(bars->kv_full[s]));
+        }
+        ++issued;
+      }
+      if (*abort_flag) {
+        // drain: wait (bounded) for the copies this thread issued that may still be landing
+        mbar_wait(bar(bars->q_full), 0, abort_flag, p.err, 0);
+        for (int j = max(0, issued - C::NS); j < issued; ++j) {
+          const unsigned long long t0 = global_timer();
+          while (!mbar_try(bar(bars->kv_full[j % C::NS]), (j / C::NS) & 1) &&
+                 global_timer() - t0 < kWaitLimitNs) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16(BM, BN, false);
+      constexpr uint32_t idesc_o = idesc_bf16(BM, D, true);
+      bool ok = mbar_wait(bar(bars->q_full), 0, abort_flag, p.err, 2);
+      tc_fence_after();
+      auto issue_pv = [&](int i) -> bool {
+        const int b = i & 1;
+        if (!mbar_wait(bar(bars->p_full[b]), (i >> 1) & 1, abort_flag, p.err, 3)) return false;
+        tc_fence_after();
+        const int s = i % C::NS;
+        const uint32_t v_base = sV + s * C::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          // B = V tile [keys][D], MN-major: 16 keys = 2 groups of 8 rows of 128 B
+          const uint64_t bd = sdesc(v_base + kk * 2048, C::ATOM_BYTES, 1024);
+          mma_ts(tmem + TM_O, tmem + TM_P + 64 * b + 8 * kk, bd, idesc_o,
+                 (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(bar(bars->pv_done[b]));
+        mma_commit(bar(bars->kv_empty[s]));
+        return true;
+      };
+      for (int j = 0; ok && j < n; ++j) {
+        const int s = j % C::NS;
+        const int b = j & 1;
+        if (!mbar_wait(bar(bars->kv_full[s]), (j / C::NS) & 1, abort_flag, p.err, 4)) break;
+        if (j >= 2 && !mbar_wait(bar(bars->s_free[b]), ((j - 2) >> 1) & 1, abort_flag, p.err, 5))
+          break;
+        tc_fence_after();
+        const uint32_t k_base = sK + s * C::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::ATOM_BYTES + (kk & 3) * 32;
+          mma_ss(tmem + TM_S + 128 * b, sdesc(sQ + off, 16, 1024), sdesc(k_base + off, 16, 1024),
+                 idesc_s, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar(bars->s_full[b]));
+        if (j >= 1 && !issue_pv(j - 1)) {
+          ok = false;
+          break;
+        }
+      }
+      if (ok && !*abort_flag && n > 0) issue_pv(n - 1);
+      // every MMA issued by this thread has completed once `drain` flips
+      mma_commit(bar(bars->drain));
+      const unsigned long long t0 = global_timer();
+      while (!mbar_try(bar(bars->drain), 0) && global_timer() - t0 < kWaitLimitNs) {
+      }
+    }
+  } else {
+    // ---------------- softmax + epilogue (warps 2..5) ----------------
+    const int quad = warp & 3;                  // TMEM lane quadrant this warp may access
+    const int row_in_tile = quad * 32 + lane;
+    const int row = q_tile * BM + row_in_tile;
+    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+    float m = -INFINITY;  // running max (log2 domain) the P values and O are relative to
+    float l = 0.f;
+    bool ok = true;
+    uint32_t S[BN];
+    for (int j = 0; j < n; ++j) {
+      const int b = j & 1;
+      // every wait in these warps is made warp-uniform, so warp-collective tcgen05 ops and
+      // votes below always run with the whole warp
+      if (!__all_sync(kFull, mbar_wait(bar(bars->s_full[b]), (j >> 1) & 1, abort_flag, p.err, 6))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < BN / 32; ++c) tmem_ld32(lane_base + TM_S + 128 * b + 32 * c, S + 32 * c);
+      tmem_wait_ld();
+      reg_fence<BN>(S);
+      tc_fence_before();
+      mbar_arrive(bar(bars->s_free[b]));
+
+      const int valid = tile_ref(p, t_begin + j).valid;
+      float mx = -INFINITY;
+      if (valid == BN) {
+#pragma unroll
+        for (int i = 0; i < BN; ++i) mx = fmaxf(mx, __uint_as_float(S[i]));
+      } else {
+#pragma unroll
+        for (int i = 0; i < BN; ++i)
+          if (i < valid) mx = fmaxf(mx, __uint_as_float(S[i]));
+      }
+      const float m_tile = mx * p.scale_log2;
+      bool rescale = false;
+      float alpha = 1.f;
+      if (m_tile > m + kRescaleThreshold) {
+        alpha = fast_exp2(m - m_tile);  // 0 on the first tile (m = -inf)
+        m = m_tile;
+        l *= alpha;
+        rescale = true;
+      }
+      // P_j goes to P[b]: PV_{j-2} must have finished reading it
+      if (j >= 2 && !__all_sync(kFull, mbar_wait(bar(bars->pv_done[b]), ((j - 2) >> 1) & 1,
+                                                 abort_flag, p.err, 7))) {
+        ok = false;
+        break;
+      }
+      const float neg_m = -m;
+#pragma unroll
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int i0 = 32 * c + 2 * i;
+          float p0 = fast_exp2(fmaf(__uint_as_float(S[i0]), p.scale_log2, neg_m));
+          float p1 = fast_exp2(fmaf(__uint_as_float(S[i0 + 1]), p.scale_log2, neg_m));
+          if (valid != BN) {
+            if (i0 >= valid) p0 = 0.f;
+            if (i0 + 1 >= valid) p1 = 0.f;
+          }
+          l += p0 + p1;
+          pk[i] = pack_bf16(p0, p1);
+        }
+        tmem_st16(lane_base + TM_P + 64 * b + 16 * c, pk);
+      }
+      if (__any_sync(0xffffffffu, rescale) && j > 0) {
+        // O holds sum_{i<j} P_i V_i relative to the old max: scale it before PV_j lands
+        if (!__all_sync(kFull, mbar_wait(bar(bars->pv_done[(j - 1) & 1]), ((j - 1) >> 1) & 1,
+                                         abort_flag, p.err, 8))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(lane_base + TM_O + 32 * c, o);
+          tmem_wait_ld();
+          reg_fence<32>(o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st16(lane_base + TM_O + 32 * c, o);
+          tmem_st16(lane_base + TM_O + 32 * c + 16, o + 16);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(bars->p_full[b]));
+    }
+    if (ok && n > 0 &&
+        __all_sync(kFull, mbar_wait(bar(bars->pv_done[(n - 1) & 1]), ((n - 1) >> 1) & 1,
+                                    abort_flag, p.err, 9))) {
+      tc_fence_after();
+      const float inv_l = 1.f / l;
+      const bool store = row < p.tokens;
+      if (p.n_splits == 1) {
+        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) +
+                             ((long long)row * p.heads + head) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(lane_base + TM_O + 32 * c, o);
+          tmem_wait_ld();
+          reg_fence<32>(o);
+          if (store) {
+            uint32_t w[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              w[i] = pack_bf16(__uint_as_float(o[2 * i]) * inv_l,
+                               __uint_as_float(o[2 * i + 1]) * inv_l);
+            uint4* dst = reinterpret_cast<uint4*>(out + 32 * c);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+          }
+        }
+      } else {
+        const long long r = ((long long)split * p.tokens + row) * p.heads + head;
+        float* po = p.part_o + r * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(lane_base + TM_O + 32 * c, o);
+          tmem_wait_ld();
+          reg_fence<32>(o);
+          if (store) {
+            float4* dst = reinterpret_cast<float4*>(po + 32 * c);
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv_l,
+                                   __uint_as_float(o[4 * v + 1]) * inv_l,
+                                   __uint_as_float(o[4 * v + 2]) * inv_l,
+                                   __uint_as_float(o[4 * v + 3]) * inv_l);
+          }
+        }
+        if (store) p.part_lse[r] = m + __log2f(l);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// out[row][h] = sum_s w_s o_s / sum_s w_s with w_s = 2^(lse_s - max_s lse_s).
+// One warp per (row, head); lane d covers features d, d+32, ... .
+template <int D>
+__global__ void __launch_bounds__(256)
+    attn_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
+                        __nv_bfloat16* __restrict__ out, int n_splits, int rows_total) {
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (gw >= rows_total) return;
+  float mx = -INFINITY;
+  for (int s = 0; s < n_splits; ++s) mx = fmaxf(mx, part_lse[(long long)s * rows_total + gw]);
+  float acc[D / 32];
+#pragma unroll
+  for (int i = 0; i < D / 32; ++i) acc[i] = 0.f;
+  float wsum = 0.f;
+  for (int s = 0; s < n_splits; ++s) {
+    const float w = exp2f(part_lse[(long long)s * rows_total + gw] - mx);
+    wsum += w;
+    const float* po = part_o + ((long long)s * rows_total + gw) * D;
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) acc[i] = fmaf(w, po[lane + 32 * i], acc[i]);
+  }
+  const float inv = 1.f / wsum;
+  __nv_bfloat16* o = out + (long long)gw * D;
+#pragma unroll
+  for (int i = 0; i < D / 32; ++i) o[lane + 32 * i] = __float2bfloat16_rn(acc[i] * inv);
+}
+
+}  // namespace
+
+size_t attn_tc_smem_bytes(int head_dim) {
+  return head_dim == 64 ? Cfg<64>::SMEM : Cfg<128>::SMEM;
+}
+
+cudaError_t launch_attn_tc(const AttnParams& p, int head_dim, int q_tiles, cudaStream_t s) {
+  dim3 grid(q_tiles, p.n_splits, p.heads);
+  cudaError_t e;
+  if (head_dim == 64) {
+    static bool attr = false;
+    if (!attr) {
+      e = cudaFuncSetAttribute(attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               Cfg<64>::SMEM);
+      if (e != cudaSuccess) return e;
+      attr = true;
+    }
+    attn_tc_kernel<64><<<grid, kThreads, Cfg<64>::SMEM, s>>>(p);
+  } else if (head_dim == 128) {
+    static bool attr = false;
+    if (!attr) {
+      e = cudaFuncSetAttribute(attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               Cfg<128>::SMEM);
+      if (e != cudaSuccess) return e;
+      attr = true;
+    }
+    attn_tc_kernel<128><<<grid, kThreads, Cfg<128>::SMEM, s>>>(p);
+  } else {
+    return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_combine(const float* part_o, const float* part_lse, void* out,
+                                int n_splits, int tokens, int heads, int head_dim,
+                                cudaStream_t s) {
+  const int rows = tokens * heads;
+  const int blocks = (rows * 32 + 255) / 256;
+  if (head_dim == 64)
+    attn_combine_kernel<64><<<blocks, 256, 0, s>>>(part_o, part_lse,
+                                                   static_cast<__nv_bfloat16*>(out), n_splits,
+                                                   rows);
+  else if (head_dim == 128)
+    attn_combine_kernel<128><<<blocks, 256, 0, s>>>(part_o, part_lse,
+                                                    static_cast<__nv_bfloat16*>(out), n_splits,
+                                                    rows);
+  else
+    return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
+}  // namespace lbm

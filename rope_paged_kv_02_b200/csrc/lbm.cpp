@@ -1,0 +1,488 @@
+// C ABI glue: RoPE table objects, the cache object (pools, scratch, tensor maps, page
+// manager) and the per-frame calls.  All validation happens here, before any state changes
+// or launches; the kernels trust their arguments.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdlib>
+#include <cstdint>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "../../include/lbm.h"
+#include "lbm_internal.h"
+#include "pager.h"
+
+struct lbm_rope {
+  lbm::RopeTables t;
+  float2* d_tables = nullptr;
+  int device = 0;
+};
+
+struct lbm_cache {
+  int heads, head_dim, patches, psi, scale_frames, sliding_window, max_frames, dtype;
+  int device = 0;
+  int num_sms = 148;
+  const lbm_rope* rope = nullptr;
+  lbm::Pools pools{};
+  void* pool_mem = nullptr;     // one allocation holding the four pools
+  float* part_o = nullptr;      // split-KV partial outputs
+  float* part_lse = nullptr;
+  int max_splits = 1;
+  int forced_splits = 0;        // LBM_ATTN_SPLITS at create time (0: planned per frame)
+  int* d_err = nullptr;
+  long long device_bytes = 0;
+  long long launches = 0;       // kernels launched so far
+  CUtensorMap tm_kp, tm_vp, tm_ks, tm_vs;
+  CUtensorMap tm_q;             // cached for the last q pointer seen
+  const void* tm_q_ptr = nullptr;
+  lbm::Pager pager;
+  cudaEvent_t ev = nullptr;     // recorded after every launch; orders calls across streams
+  cudaStream_t last_stream = nullptr;
+  bool ev_valid = false;
+  lbm_cache(int s, int w, int m, int psi_) : pager(s, w, m, psi_) {}
+};
+
+namespace {
+
+constexpr int kMaxSplits = 16;
+
+int elem_size(int dtype) { return dtype == LBM_BF16 ? 2 : 4; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 3-D bf16 tensor map {d0 (contiguous), d1, d2} with strides (bytes) s1, s2 and box
+// {64, b1, b2}, 128-byte swizzle, zero fill out of bounds.
+bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+              uint64_t s1, uint64_t s2, uint32_t b1, uint32_t b2) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {s1, s2};
+  cuuint32_t box[3] = {64, b1, b2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+int use_device(int dev) {
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess) return LBM_ERR_CUDA;
+  if (cur != dev && cudaSetDevice(dev) != cudaSuccess) return LBM_ERR_CUDA;
+  return LBM_OK;
+}
+
+void order_before(lbm_cache* c, cudaStream_t s) {
+  if (c->ev_valid && s != c->last_stream) cudaStreamWaitEvent(s, c->ev, 0);
+}
+
+void order_after(lbm_cache* c, cudaStream_t s) {
+  cudaEventRecord(c->ev, s);
+  c->last_stream = s;
+  c->ev_valid = true;
+}
+
+// Number of key splits: minimise waves x (tiles per split + fixed cost) + combine cost.
+int plan_splits(int work_units, int n_tiles, int num_sms, double combine_tiles_per_split,
+                int max_splits) {
+  int best = 1;
+  double best_cost = 1e30;
+  const int lim = n_tiles < max_splits ? n_tiles : max_splits;
+  for (int s = 1; s <= lim; ++s) {
+    const int tps = (n_tiles + s - 1) / s;
+    const int s_eff = (n_tiles + tps - 1) / tps;
+    if (s_eff != s) continue;
+    const long long units = (long long)work_units * s;
+    const long long waves = (units + num_sms - 1) / num_sms;
+    double cost = (double)waves * (tps + 6.0);
+    if (s > 1) cost += 8.0 + combine_tiles_per_split * s;
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = s;
+    }
+  }
+  return best;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* lbm_status_string(int status) {
+  switch (status) {
+    case LBM_OK: return "ok";
+    case LBM_ERR_INVALID: return "invalid argument";
+    case LBM_ERR_UNSUPPORTED: return "unsupported configuration";
+    case LBM_ERR_SEQUENCE: return "call out of sequence";
+    case LBM_ERR_CAPACITY: return "capacity exceeded";
+    case LBM_ERR_NOMEM: return "out of memory";
+    case LBM_ERR_CUDA: return "CUDA error";
+    case LBM_ERR_TIMEOUT: return "device wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int lbm_rope3d_tables(int head_dim, int ppf, int pph, int ppw, int patch_start_idx,
+                      double theta, lbm_rope_t** out) {
+  if (!out) return LBM_ERR_INVALID;
+  *out = nullptr;
+  if (head_dim < 6 || head_dim % 2 || ppf < 1 || pph < 1 || ppw < 1 || patch_start_idx < 0 ||
+      !(theta > 1.0) || (long long)pph * ppw > (1 << 20) || ppf > (1 << 24))
+    return LBM_ERR_INVALID;
+  // Axis split: d_h = d_w = 2 * (head_dim / 6), d_t = the rest; pairs ordered t, h, w.
+  const int dh = 2 * (head_dim / 6);
+  const int dt = head_dim - 2 * dh;
+  lbm::RopeTables t{};
+  t.head_dim = head_dim;
+  t.ppf = ppf;
+  t.pph = pph;
+  t.ppw = ppw;
+  t.psi = patch_start_idx;
+  t.nt = dt / 2;
+  t.nh = dh / 2;
+  t.nw = dh / 2;
+  const size_t n_t = (size_t)ppf * t.nt, n_h = (size_t)(pph + 1) * t.nh,
+               n_w = (size_t)(ppw + 1) * t.nw;
+  std::vector<float2> host(n_t + n_h + n_w);
+  // angle(p, i) = p * theta^(-2i/d_axis), in double, cos/sin rounded once to float
+  auto fill = [&](float2* dst, int rows, int pairs, int d_axis) {
+    for (int i = 0; i < pairs; ++i) {
+      const double inv = std::pow(theta, -(2.0 * i) / (double)d_axis);
+      for (int p = 0; p < rows; ++p) {
+        const double a = (double)p * inv;
+        dst[(size_t)p * pairs + i] = make_float2((float)std::cos(a), (float)std::sin(a));
+      }
+    }
+  };
+  fill(host.data(), ppf, t.nt, dt);
+  fill(host.data() + n_t, pph + 1, t.nh, dh);
+  fill(host.data() + n_t + n_h, ppw + 1, t.nw, dh);
+  auto* r = new (std::nothrow) lbm_rope;
+  if (!r) return LBM_ERR_NOMEM;
+  if (cudaGetDevice(&r->device) != cudaSuccess ||
+      cudaMalloc(&r->d_tables, host.size() * sizeof(float2)) != cudaSuccess) {
+    delete r;
+    cudaGetLastError();
+    return LBM_ERR_NOMEM;
+  }
+  if (cudaMemcpy(r->d_tables, host.data(), host.size() * sizeof(float2),
+                 cudaMemcpyHostToDevice) != cudaSuccess) {
+    cudaFree(r->d_tables);
+    delete r;
+    return LBM_ERR_CUDA;
+  }
+  t.tab_t = r->d_tables;
+  t.tab_h = r->d_tables + n_t;
+  t.tab_w = r->d_tables + n_t + n_h;
+  r->t = t;
+  *out = r;
+  return LBM_OK;
+}
+
+int lbm_rope3d_expand(const lbm_rope_t* rope, float* cos_out, float* sin_out, void* stream) {
+  if (!rope || !cos_out || !sin_out) return LBM_ERR_INVALID;
+  if (use_device(rope->device) != LBM_OK) return LBM_ERR_CUDA;
+  return lbm::launch_rope_expand(rope->t, cos_out, sin_out, (cudaStream_t)stream) == cudaSuccess
+             ? LBM_OK
+             : LBM_ERR_CUDA;
+}
+
+void lbm_rope_destroy(lbm_rope_t* rope) {
+  if (!rope) return;
+  cudaFree(rope->d_tables);
+  delete rope;
+}
+
+int lbm_cache_create(int heads, int head_dim, int patches_per_frame, int specials_per_frame,
+                     int scale_frames, int sliding_window, int max_frames, int dtype,
+                     const lbm_rope_t* rope, lbm_cache_t** out) {
+  if (!out) return LBM_ERR_INVALID;
+  *out = nullptr;
+  if (!rope || heads < 1 || heads > 65535 || patches_per_frame < 1 || scale_frames < 0 ||
+      sliding_window < 0 || max_frames < 1 ||
+      scale_frames + sliding_window + 1 > LBM_MAX_PAGES)
+    return LBM_ERR_INVALID;
+  if (dtype != LBM_BF16 && dtype != LBM_F32) return LBM_ERR_UNSUPPORTED;
+  if (head_dim != 64 && head_dim != 128) return LBM_ERR_UNSUPPORTED;
+  if (specials_per_frame != 6 || rope->t.psi != specials_per_frame ||
+      rope->t.head_dim != head_dim || rope->t.pph * rope->t.ppw != patches_per_frame)
+    return LBM_ERR_INVALID;
+
+  auto* c = new (std::nothrow) lbm_cache(scale_frames, sliding_window, max_frames, 6);
+  if (!c) return LBM_ERR_NOMEM;
+  c->heads = heads;
+  c->head_dim = head_dim;
+  c->patches = patches_per_frame;
+  c->psi = specials_per_frame;
+  c->scale_frames = scale_frames;
+  c->sliding_window = sliding_window;
+  c->max_frames = max_frames;
+  c->dtype = dtype;
+  c->rope = rope;
+  cudaGetDevice(&c->device);
+  cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device);
+  if (const char* env = std::getenv("LBM_ATTN_SPLITS")) {
+    const int v = std::atoi(env);
+    if (v >= 1 && v <= kMaxSplits) c->forced_splits = v;
+  }
+
+  const int P = scale_frames + sliding_window + 1;
+  const int stride = (patches_per_frame + 127) / 128 * 128;
+  const long long cap = (6LL * (max_frames + 1) + 127) / 128 * 128;
+  const int e = elem_size(dtype);
+  const size_t patch_bytes = (size_t)heads * P * stride * head_dim * e;
+  const size_t spec_bytes = (size_t)heads * cap * head_dim * e;
+  const size_t total = 2 * patch_bytes + 2 * spec_bytes;
+  const int T = specials_per_frame + patches_per_frame;
+  c->max_splits = dtype == LBM_BF16 ? kMaxSplits : 1;
+  const size_t part_o_bytes = (size_t)c->max_splits * T * heads * head_dim * sizeof(float);
+  const size_t part_lse_bytes = (size_t)c->max_splits * T * heads * sizeof(float);
+  auto fail = [&](int st) {
+    cudaFree(c->pool_mem);
+    cudaFree(c->part_o);
+    cudaFree(c->part_lse);
+    cudaFree(c->d_err);
+    if (c->ev) cudaEventDestroy(c->ev);
+    cudaGetLastError();
+    delete c;
+    return st;
+  };
+  if (cap > (1LL << 31) / 2) return fail(LBM_ERR_INVALID);
+  if (cudaMalloc(&c->pool_mem, total) != cudaSuccess) return fail(LBM_ERR_NOMEM);
+  if (cudaMemset(c->pool_mem, 0, total) != cudaSuccess) return fail(LBM_ERR_CUDA);
+  if (dtype == LBM_BF16) {
+    if (cudaMalloc(&c->part_o, part_o_bytes) != cudaSuccess ||
+        cudaMalloc(&c->part_lse, part_lse_bytes) != cudaSuccess)
+      return fail(LBM_ERR_NOMEM);
+  }
+  if (cudaMalloc(&c->d_err, sizeof(int)) != cudaSuccess) return fail(LBM_ERR_NOMEM);
+  if (cudaMemset(c->d_err, 0, sizeof(int)) != cudaSuccess) return fail(LBM_ERR_CUDA);
+  if (cudaEventCreateWithFlags(&c->ev, cudaEventDisableTiming) != cudaSuccess)
+    return fail(LBM_ERR_CUDA);
+  char* base = static_cast<char*>(c->pool_mem);
+  c->pools.k_patch = base;
+  c->pools.v_patch = base + patch_bytes;
+  c->pools.k_special = base + 2 * patch_bytes;
+  c->pools.v_special = base + 2 * patch_bytes + spec_bytes;
+  c->pools.num_pages = P;
+  c->pools.page_stride = stride;
+  c->pools.spec_cap = (int)cap;
+  c->device_bytes = (long long)(total + (dtype == LBM_BF16 ? part_o_bytes + part_lse_bytes : 0) +
+                                sizeof(int));
+  if (dtype == LBM_BF16) {
+    const uint64_t row = (uint64_t)head_dim * 2;
+    const uint64_t prow = (uint64_t)P * stride;
+    if (!make_map(&c->tm_kp, c->pools.k_patch, head_dim, prow, heads, row, prow * row, 128, 1) ||
+        !make_map(&c->tm_vp, c->pools.v_patch, head_dim, prow, heads, row, prow * row, 128, 1) ||
+        !make_map(&c->tm_ks, c->pools.k_special, head_dim, cap, heads, row, cap * row, 128, 1) ||
+        !make_map(&c->tm_vs, c->pools.v_special, head_dim, cap, heads, row, cap * row, 128, 1))
+      return fail(LBM_ERR_CUDA);
+  }
+  if (cudaDeviceSynchronize() != cudaSuccess) return fail(LBM_ERR_CUDA);
+  *out = c;
+  return LBM_OK;
+}
+
+int lbm_append_frame(lbm_cache_t* c, void* q, const void* k, const void* v, long long frame_idx,
+                     int is_keyframe, void* stream) {
+  if (!c || !q || !k || !v || !aligned16(q) || !aligned16(k) || !aligned16(v))
+    return LBM_ERR_INVALID;
+  if (frame_idx < 0 || frame_idx >= c->rope->t.ppf) return LBM_ERR_SEQUENCE;
+  int page = -1, slot = -1;
+  switch (c->pager.peek_append(frame_idx, is_keyframe != 0, &page, &slot)) {
+    case lbm::PagerStatus::kOk: break;
+    case lbm::PagerStatus::kSequence: return LBM_ERR_SEQUENCE;
+    case lbm::PagerStatus::kCapacity: return LBM_ERR_CAPACITY;
+  }
+  if (use_device(c->device) != LBM_OK) return LBM_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  lbm::AppendArgs a{};
+  a.dtype = c->dtype;
+  a.heads = c->heads;
+  a.head_dim = c->head_dim;
+  a.tokens = c->psi + c->patches;
+  a.psi = c->psi;
+  a.frame = (int)frame_idx;
+  a.page = page;
+  a.special_slot = slot;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  order_before(c, s);
+  if (lbm::launch_rope_append(c->rope->t, c->pools, a, s) != cudaSuccess) return LBM_ERR_CUDA;
+  ++c->launches;
+  order_after(c, s);
+  c->pager.append(frame_idx, is_keyframe != 0, &page, &slot);
+  return LBM_OK;
+}
+
+int lbm_attend_frame(lbm_cache_t* c, const void* q, void* out, void* stream) {
+  if (!c || !q || !out || !aligned16(q) || !aligned16(out)) return LBM_ERR_INVALID;
+  std::vector<int> pages;
+  int n_sp = 0, last_len = 0;
+  if (c->pager.visible(&pages, &n_sp, &last_len) != lbm::PagerStatus::kOk)
+    return LBM_ERR_SEQUENCE;
+  if (use_device(c->device) != LBM_OK) return LBM_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int T = c->psi + c->patches;
+  order_before(c, s);
+  if (c->dtype == LBM_BF16) {
+    static thread_local lbm::AttnParams p;  // ~3 KB: kept off the stack
+    if (q != c->tm_q_ptr) {
+      const uint64_t row = (uint64_t)c->head_dim * 2;
+      if (!make_map(&c->tm_q, q, c->head_dim, c->heads, T, row, row * c->heads, 1, 128))
+        return LBM_ERR_CUDA;
+      c->tm_q_ptr = q;
+    }
+    p.tm_q = c->tm_q;
+    p.tm_kp = c->tm_kp;
+    p.tm_vp = c->tm_vp;
+    p.tm_ks = c->tm_ks;
+    p.tm_vs = c->tm_vs;
+    p.out = out;
+    p.part_o = c->part_o;
+    p.part_lse = c->part_lse;
+    p.err = c->d_err;
+    p.tokens = T;
+    p.heads = c->heads;
+    p.patches = c->patches;
+    p.page_stride = c->pools.page_stride;
+    p.tiles_per_page = c->pools.page_stride / 128;
+    p.n_pages = (int)pages.size();
+    p.n_special = n_sp;
+    p.n_tiles = p.n_pages * p.tiles_per_page + (n_sp + 127) / 128;
+    p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)c->head_dim));
+    for (size_t i = 0; i < pages.size(); ++i) p.pages[i] = (uint16_t)pages[i];
+    const int q_tiles = (T + 127) / 128;
+    const double combine = (double)T * c->heads * c->head_dim * 4.0 / 1.8e6;
+    p.n_splits = plan_splits(q_tiles * c->heads, p.n_tiles, c->num_sms, combine, c->max_splits);
+    if (c->forced_splits) p.n_splits = std::min(c->forced_splits, p.n_tiles);
+    p.tiles_per_split = (p.n_tiles + p.n_splits - 1) / p.n_splits;
+    p.n_splits = (p.n_tiles + p.tiles_per_split - 1) / p.tiles_per_split;  // no empty split
+    if (lbm::launch_attn_tc(p, c->head_dim, q_tiles, s) != cudaSuccess) return LBM_ERR_CUDA;
+    ++c->launches;
+    if (p.n_splits > 1) {
+      if (lbm::launch_attn_combine(c->part_o, c->part_lse, out, p.n_splits, T, c->heads,
+                                   c->head_dim, s) != cudaSuccess)
+        return LBM_ERR_CUDA;
+      ++c->launches;
+    }
+  } else {
+    static thread_local lbm::SimtParams p;
+    p.q = q;
+    p.out = out;
+    p.k_patch = c->pools.k_patch;
+    p.v_patch = c->pools.v_patch;
+    p.k_special = c->pools.k_special;
+    p.v_special = c->pools.v_special;
+    p.tokens = T;
+    p.heads = c->heads;
+    p.head_dim = c->head_dim;
+    p.patches = c->patches;
+    p.page_stride = c->pools.page_stride;
+    p.pool_pages = c->pools.num_pages;
+    p.spec_cap = c->pools.spec_cap;
+    p.n_pages = (int)pages.size();
+    p.n_special = n_sp;
+    p.scale = (float)(1.0 / std::sqrt((double)c->head_dim));
+    for (size_t i = 0; i < pages.size(); ++i) p.pages[i] = (uint16_t)pages[i];
+    if (lbm::launch_attn_simt(p, s) != cudaSuccess) return LBM_ERR_CUDA;
+    ++c->launches;
+  }
+  order_after(c, s);
+  int evicted = -1;
+  c->pager.finish(&evicted);
+  return LBM_OK;
+}
+
+int lbm_cache_reset(lbm_cache_t* c) {
+  if (!c) return LBM_ERR_INVALID;
+  c->pager.reset();
+  return LBM_OK;
+}
+
+int lbm_cache_state(const lbm_cache_t* c, lbm_cache_state_t* st) {
+  if (!c || !st) return LBM_ERR_INVALID;
+  st->device_bytes = c->device_bytes;
+  st->kernel_launches = c->launches;
+  return lbm::fill_state(c->pager, st);
+}
+
+int lbm_cache_read_kv(const lbm_cache_t* c, int which, int index, int count, void* host_out) {
+  if (!c || !host_out) return LBM_ERR_INVALID;
+  const int e = elem_size(c->dtype);
+  const size_t row = (size_t)c->head_dim * e;
+  const void* src;
+  size_t pitch, width;
+  if (which == LBM_K_PATCH || which == LBM_V_PATCH) {
+    if (index < 0 || index >= c->pools.num_pages) return LBM_ERR_INVALID;
+    const char* pool = static_cast<const char*>(which == LBM_K_PATCH ? c->pools.k_patch
+                                                                     : c->pools.v_patch);
+    src = pool + (size_t)index * c->pools.page_stride * row;
+    pitch = (size_t)c->pools.num_pages * c->pools.page_stride * row;
+    width = (size_t)c->patches * row;
+  } else if (which == LBM_K_SPECIAL || which == LBM_V_SPECIAL) {
+    if (index < 0 || count < 1 || index + count > c->pools.spec_cap) return LBM_ERR_INVALID;
+    const char* pool = static_cast<const char*>(which == LBM_K_SPECIAL ? c->pools.k_special
+                                                                       : c->pools.v_special);
+    src = pool + (size_t)index * row;
+    pitch = (size_t)c->pools.spec_cap * row;
+    width = (size_t)count * row;
+  } else {
+    return LBM_ERR_INVALID;
+  }
+  if (use_device(c->device) != LBM_OK) return LBM_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return LBM_ERR_CUDA;
+  if (cudaMemcpy2D(host_out, width, src, pitch, width, c->heads, cudaMemcpyDeviceToHost) !=
+      cudaSuccess)
+    return LBM_ERR_CUDA;
+  return LBM_OK;
+}
+
+int lbm_cache_check(lbm_cache_t* c) {
+  if (!c) return LBM_ERR_INVALID;
+  if (use_device(c->device) != LBM_OK) return LBM_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return LBM_ERR_CUDA;
+  int err = 0;
+  if (cudaMemcpy(&err, c->d_err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return LBM_ERR_CUDA;
+  if (err != 0) {
+    cudaMemset(c->d_err, 0, sizeof(int));
+    return LBM_ERR_TIMEOUT;
+  }
+  return LBM_OK;
+}
+
+void lbm_cache_destroy(lbm_cache_t* c) {
+  if (!c) return;
+  use_device(c->device);
+  cudaDeviceSynchronize();
+  cudaFree(c->pool_mem);
+  cudaFree(c->part_o);
+  cudaFree(c->part_lse);
+  cudaFree(c->d_err);
+  if (c->ev) cudaEventDestroy(c->ev);
+  delete c;
+}
+
+}  // extern "C"

@@ -1,0 +1,207 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle on seeded inputs.
+
+Steps checked per frame (tolerances in ``tests/stream_check.py``): the 3D RoPE of q (in
+place) and of k, the pages and special slots written by the fused rotate+append kernel,
+the page table / free list / retained frames (bit-exact) and the paged attention output.
+"""
+
+import os
+
+import numpy as np
+import pytest
+
+from oracle import rope3d
+from rope_paged_kv_02_b200 import _lib
+from rope_paged_kv_02_b200.workloads import CONFIGS, custom_config
+
+from stream_check import run_stream
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from rope_paged_kv_02_b200.build import build
+    build()
+    _lib.load()
+
+
+@pytest.mark.parametrize("head_dim,ppf,pph,ppw", [(64, 30, 14, 14), (128, 5, 64, 64),
+                                                  (64, 2000, 37, 27)])
+def test_rope_tables_match_oracle(head_dim, ppf, pph, ppw):
+    import torch
+    rope = _lib.Rope3D(head_dim, ppf, pph, ppw, 6)
+    rows = ppf * (6 + pph * ppw)
+    cos = torch.empty(rows, head_dim // 2, device="cuda")
+    sin = torch.empty_like(cos)
+    rope.expand(cos, sin)
+    torch.cuda.synchronize()
+    ec, es = rope3d.expanded_table(head_dim, ppf, pph, ppw, 6)
+    assert np.abs(cos.cpu().numpy() - ec).max() <= 1e-5
+    assert np.abs(sin.cpu().numpy() - es).max() <= 1e-5
+    rope.close()
+
+
+def test_tiny_fp32_config_all_frames():
+    run_stream(CONFIGS[0])
+
+
+SMALL = [
+    # two query tiles with a ragged tail, two key tiles per page (130 patches), keyframe
+    # every 2nd frame (rollbacks)
+    custom_config(200, 2, 64, "bf16", 10, 13, 9, 2, 1, 2),
+    # head_dim 128, odd patch count, keyframe every 3rd frame
+    custom_config(201, 2, 128, "bf16", 9, 15, 12, 3, 2, 1),
+    # T = 22 < 128; no scale frames; specials cross the 128-token special page at frame 21
+    custom_config(202, 3, 64, "bf16", 4, 4, 40, 1, 0, 3),
+    # no sliding window: every frame after the scale frames is evicted right after attending
+    custom_config(203, 1, 64, "bf16", 6, 6, 6, 1, 2, 0),
+    # fp32 cache, head_dim 128
+    custom_config(204, 2, 128, "f32", 3, 5, 7, 2, 1, 2),
+]
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
+def test_small_streams_all_frames_all_rows(cfg):
+    run_stream(cfg)
+
+
+@pytest.mark.parametrize("splits", ["1", "3", "16"])
+def test_forced_split_counts_agree(splits, monkeypatch):
+    monkeypatch.setenv("LBM_ATTN_SPLITS", splits)
+    run_stream(custom_config(205, 2, 64, "bf16", 12, 12, 8, 1, 2, 3))
+
+
+def test_non_contiguous_frame_indices():
+    cfg = custom_config(206, 2, 64, "bf16", 5, 7, 8, 2, 1, 2)
+    run_stream(cfg, frame_ids=[0, 3, 4, 10, 11, 20, 57, 58])
+
+
+def _needle(cfg, n_needle_frame, target_frame, row, boost):
+    """Tamper hook: plant at frame n_needle_frame a key equal to boost * (rotated q of
+    target_frame, row), and scale every q by 4 (peaked softmax: scores of std 4, the
+    needle's about 25)."""
+    from rope_paged_kv_02_b200.workloads import frame_qkv, round_bf16
+    q_t, _, _ = frame_qkv(cfg, target_frame)
+    q_rot = rope3d.rotate_frame(q_t.astype(np.float64) * 4.0, target_frame, 6, cfg.pph, cfg.ppw)
+    slot = 6 + 5
+    pos = rope3d.token_positions(n_needle_frame, 6, cfg.pph, cfg.ppw)[slot:slot + 1]
+    kneedle = rope3d.rotate(boost * q_rot[row:row + 1],
+                            -rope3d.angles_for_positions(pos, cfg.head_dim))[0]
+
+    def tamper(n, q, k, v):
+        q = q * np.float32(4.0)       # exact in bf16 and fp32
+        if n == n_needle_frame:
+            k = k.copy()
+            k[slot] = round_bf16(kneedle.astype(np.float32)) if cfg.dtype == "bf16" else kneedle
+        return q, k, v
+
+    return tamper
+
+
+def test_peaked_softmax_with_needle_key():
+    cfg = custom_config(207, 2, 64, "bf16", 10, 13, 6, 1, 1, 3)
+    tamper = _needle(cfg, 2, 5, 0, 0.2)
+    run_stream(cfg, tamper=tamper)
+
+
+@pytest.mark.parametrize("cid,frames", [
+    (1, [0, 1, 8, 24, 25, 63]),
+    (2, [0, 4, 5, 315, 316, 319]),
+    (4, [0, 36, 37, 95]),
+])
+def test_full_size_config_sampled(cid, frames):
+    cfg = CONFIGS[cid]
+    rng = np.random.default_rng(cid)
+    rows = np.unique(np.concatenate([np.arange(6), [cfg.tokens - 1],
+                                     rng.choice(cfg.tokens, 120, replace=False)]))
+    run_stream(cfg, check_frames=frames, rows=rows, regenerate=True)
+
+
+@pytest.mark.slow
+def test_long_stream_2000_keyframes_sampled():
+    cfg = CONFIGS[3]
+    rng = np.random.default_rng(3)
+    rows = np.unique(np.concatenate([np.arange(6), [cfg.tokens - 1],
+                                     rng.choice(cfg.tokens, 58, replace=False)]))
+    run_stream(cfg, check_frames=[0, 135, 136, 137, 1000, 1999], rows=rows, regenerate=True,
+               check_pools=False)
+
+
+def test_sequence_errors_leave_state_unchanged():
+    import torch
+    cfg = custom_config(208, 2, 64, "bf16", 4, 4, 4, 1, 1, 1)
+    rope = _lib.Rope3D(64, 4, 4, 4, 6)
+    cache = _lib.PagedKVCache(rope, 2, 64, 16, 1, 1, 2, _lib.LBM_BF16)
+    q = torch.randn(22, 2, 64, device="cuda").to(torch.bfloat16)
+    k, v, out = torch.randn_like(q), torch.randn_like(q), torch.empty_like(q)
+    with pytest.raises(_lib.LbmError) as e:
+        cache.attend_frame(q, out)                        # nothing appended
+    assert e.value.status == _lib.LBM_ERR_SEQUENCE
+    cache.append_frame(q, k, v, 0, True)
+    s0 = cache.state()
+    with pytest.raises(_lib.LbmError) as e:
+        cache.append_frame(q, k, v, 1, True)              # append twice
+    assert e.value.status == _lib.LBM_ERR_SEQUENCE
+    assert cache.state() == s0
+    cache.attend_frame(q, out)
+    with pytest.raises(_lib.LbmError) as e:
+        cache.append_frame(q, k, v, 4, True)              # beyond the t table (ppf = 4)
+    assert e.value.status == _lib.LBM_ERR_SEQUENCE
+    with pytest.raises(_lib.LbmError) as e:
+        cache.append_frame(q, k, v, 0, True)              # frame index must increase
+    assert e.value.status == _lib.LBM_ERR_SEQUENCE
+    bad = q.view(-1)[1:].view(-1)                         # 2-byte offset: misaligned
+    with pytest.raises(_lib.LbmError) as e:
+        cache.append_frame(bad, k, v, 1, True)
+    assert e.value.status == _lib.LBM_ERR_INVALID
+    cache.append_frame(q, k, v, 1, True)
+    cache.attend_frame(q, out)
+    s1 = cache.state()
+    with pytest.raises(_lib.LbmError) as e:
+        cache.append_frame(q, k, v, 2, True)              # max_frames = 2 keyframes held
+    assert e.value.status == _lib.LBM_ERR_CAPACITY
+    assert cache.state() == s1
+    cache.append_frame(q, k, v, 2, False)                 # a non-keyframe still fits
+    cache.attend_frame(q, out)
+    cache.check()
+    cache.reset()
+    st = cache.state()
+    assert st["free"] == [2, 1, 0] and st["n_special"] == 0 and not st["pending"]
+    with pytest.raises(_lib.LbmError) as e:
+        _lib.PagedKVCache(rope, 2, 96, 16, 1, 1, 2, _lib.LBM_BF16)
+    assert e.value.status == _lib.LBM_ERR_UNSUPPORTED
+    with pytest.raises(_lib.LbmError) as e:
+        _lib.PagedKVCache(rope, 2, 64, 15, 1, 1, 2, _lib.LBM_BF16)   # != pph * ppw
+    assert e.value.status == _lib.LBM_ERR_INVALID
+    cache.close()
+    rope.close()
+
+
+def test_calls_on_two_streams_are_ordered():
+    """append on one stream, attend on another: the library orders them with its event."""
+    import torch
+    cfg = custom_config(209, 2, 64, "bf16", 8, 8, 6, 1, 1, 2)
+    from rope_paged_kv_02_b200.workloads import frame_qkv
+    from oracle import stream as ostream
+    from stream_check import check_attn, dev, host
+    rope = _lib.Rope3D(64, 6, 8, 8, 6)
+    cache = _lib.PagedKVCache(rope, 2, 64, 64, 1, 2, 6, _lib.LBM_BF16)
+    so = ostream.StreamOracle(2, 64, 8, 8, 1, 2, 6)
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    for f in range(6):
+        q, k, v = frame_qkv(cfg, f)
+        with torch.cuda.stream(s1):
+            qd, kd, vd = dev(q, "bf16"), dev(k, "bf16"), dev(v, "bf16")
+            out = torch.empty_like(qd)
+            cache.append_frame(qd, kd, vd, f, True, stream=s1)
+        s2.wait_stream(s1)    # the caller orders its own buffers; the cache orders itself
+        cache.attend_frame(qd, out, stream=s2)
+        torch.cuda.synchronize()
+        r = so.step(f, True, q, k, v)
+        check_attn(host(out), r.out, f"frame {f}")
+    cache.close()
+    rope.close()

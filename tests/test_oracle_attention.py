@@ -68,7 +68,7 @@ def test_attention_properties():
                                atol=1e-13)                                   # key order
     rows = [0, 3, 6]
     np.testing.assert_allclose(attention.attend(q[rows], k, v), attention.attend(q, k, v)[rows],
-                               atol=0)                                       # rows independent
+                               atol=1e-14, rtol=0)                           # rows independent
 
 
 @pytest.mark.parametrize("cfg", [CONFIGS[0],
@@ -130,3 +130,22 @@ def test_needle_key_is_found_in_its_page():
     r, needle_v = _needle_stream(2)           # frame 2 evicted before frame 5
     assert r.visible_frames == [0, 3, 4, 5]
     assert np.abs(r.out[0, 0] - needle_v).max() > 0.1
+
+
+def test_regenerated_kv_source_matches_stored_kv():
+    """The long-stream mode (retained keys re-created from the seeded inputs) agrees exactly."""
+    cfg = custom_config(104, 2, 64, "bf16", 3, 4, 15, 2, 1, 3)
+
+    def source(frame, region):
+        q, k, v = frame_qkv(cfg, frame)
+        sl = slice(6, None) if region == "patch" else slice(0, 6)
+        return k[sl], v[sl]
+
+    a = stream.StreamOracle(2, 64, 3, 4, 1, 3, cfg.n_keyframes)
+    b = stream.StreamOracle(2, 64, 3, 4, 1, 3, cfg.n_keyframes, kv_source=source)
+    for f, key in enumerate(cfg.keyframes):
+        q, k, v = frame_qkv(cfg, f)
+        ra = a.step(f, key, q, k, v)
+        rb = b.step(f, key, q, k, v, rows=[0, 5, 7, 17])
+        np.testing.assert_allclose(rb.out, ra.out[[0, 5, 7, 17]], atol=1e-13, rtol=0)
+        assert ra.state == rb.state
