@@ -5,20 +5,24 @@
 // over the visible page table (scale pages -> window pages -> own page -> special pages,
 // the last special page partly filled), with K/V that already carry their rotation.
 //
-// One CTA = one (query tile of 128 rows, split of the key tiles, head).  Warp roles:
-//   warp 0      TMA producer: Q tile once, then K/V tiles gathered page by page through
-//               the page table into a ring of shared-memory stages (128B swizzle).
-//   warp 1      allocates tensor memory; one lane issues every tcgen05.mma:
-//                 S_j = Q K_j^T   (A, B from shared memory)      -> TMEM S[j%2]
-//                 O  += P_j V_j   (A = P from TMEM, B = V smem)   -> TMEM O
-//               S_{j+1} is issued before waiting for P_j, so the tensor core works on the
-//               next scores while the softmax warps work on this tile.
-//   warps 2..5  softmax: each thread owns one query row (its TMEM lane); reads S_j,
-//               row max, exp2, row sum in fp32, writes P_j (bf16) into TMEM, and
-//               rescales O only when the running max grew by more than 2^8 (lazy
-//               rescale; exact because O and l always share the same reference max).
-// Tensor memory (512 columns): S0 [0,128) S1 [128,256) P0 [256,320) P1 [320,384)
-// O [384, 384+D).
+// One CTA = two query tiles of 128 rows of one head, over one split of the key tiles.
+// Both query tiles share every K/V tile the CTA loads.  Warp roles (12 warps):
+//   warp 0      TMA producer: the two Q tiles once, then K/V tiles gathered page by page
+//               through the page table into a ring of shared-memory stages (128B swizzle).
+//   warp 1, 2   allocate tensor memory (warp 1); one lane of warp 1+g issues every
+//               tcgen05.mma of query tile g:
+//                 S = Q_g K_j^T   (A, B from shared memory)      -> TMEM S_g
+//                 O_g += P V_j    (A = P from TMEM, B = V smem)   -> TMEM O_g
+//               With head_dim 64, S_{j+1} is issued as soon as the softmax warps have read
+//               S_j, before PV_j, so scores and softmax overlap.
+//   warps 4..7  softmax of query tile 0, warps 8..11 of tile 1: each thread owns one query
+//               row (its TMEM lane); reads S_j, row max, exp2, row sum in fp32, writes P_j
+//               (bf16) into TMEM, and rescales O only when the running max grew by more than
+//               2^8 (lazy rescale; exact because O and l share one reference max).
+//   The two softmax warpgroups run concurrently, so one's exponentials overlap the other's
+//   tensor-core work.
+// Tensor memory: 256 columns per query tile g at 256 g: S [0,128); head_dim 64:
+// P [128,192), O [192,256); head_dim 128: O [128,256), P written over S [0,64).
 // Every mbarrier wait is bounded (about 2 s); a wait that runs out sets the device error
 // word, raises a CTA-wide abort flag, and every role falls through to the common exit,
 // which drains outstanding copies / MMAs (bounded) and frees tensor memory.
@@ -32,23 +36,20 @@ namespace {
 
 constexpr int BM = 128;         // query rows per CTA
 constexpr int BN = 128;         // keys per tile
-constexpr int kThreads = 192;   // 6 warps
+constexpr int kThreads = 384;   // 12 warps
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t TM_S = 0;    // S buffer b at TM_S + 128 b
-constexpr uint32_t TM_P = 256;  // P buffer b at TM_P + 64 b
-constexpr uint32_t TM_O = 384;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when max grows by > 2^8
 constexpr unsigned kFull = 0xffffffffu;
 
 template <int D>
 struct Cfg {
-  static constexpr int NS = D == 64 ? 4 : 3;            // K/V pipeline stages
+  static constexpr int NS = D == 64 ? 4 : 2;            // K/V pipeline stages
   static constexpr int ATOM_BYTES = 128 * 128;          // 128 rows x 64 bf16 (one swizzle atom column)
   static constexpr int ATOMS = D / 64;
   static constexpr int TILE_BYTES = ATOMS * ATOM_BYTES; // one Q, K or V tile
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + TILE_BYTES;
+  static constexpr int OFF_Q = 0;                       // two query tiles
+  static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
   static constexpr int OFF_V = OFF_K + NS * TILE_BYTES;
   static constexpr int OFF_BAR = OFF_V + NS * TILE_BYTES;
   static constexpr int BAR_BYTES = 256;
@@ -239,22 +240,34 @@ __device__ __forceinline__ TileRef tile_ref(const AttnParams& p, int t) {
 }
 
 struct Bars {
-  uint64_t q_full;
-  uint64_t s_full[2];
-  uint64_t s_free[2];
-  uint64_t p_full[2];
-  uint64_t pv_done[2];
-  uint64_t drain;
+  uint64_t q_full[2];
+  uint64_t s_full[2];    // per query tile g: S_j landed in TMEM
+  uint64_t s_free[2];    // per g: the softmax warps have read S_j
+  uint64_t p_full[2];    // per g: P_j written to TMEM (and O rescaled if needed)
+  uint64_t pv_done[2];   // per g: PV_j finished (P buffer and O are free again)
+  uint64_t drain[2];
   uint64_t kv_full[4];
-  uint64_t kv_empty[4];
+  uint64_t kv_empty[4];  // one arrival per active query tile
   uint32_t tmem_base;
   int abort_flag;
+};
+
+// Per-tile softmax state of one query row, and the TMEM column map of query tile g.
+template <int D>
+struct TmemMap {
+  // 256 columns per query tile: S [0,128); D = 64: P [128,192), O [192,256);
+  // D = 128: O [128,256) and P overwrites S [0,64) once S has been read into registers.
+  static constexpr uint32_t S = 0;
+  static constexpr uint32_t P = D == 64 ? 128 : 0;
+  static constexpr uint32_t O = D == 64 ? 192 : 128;
+  static constexpr bool kPAliasesS = D != 64;
 };
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ AttnParams p) {
   using C = Cfg<D>;
+  using TM = TmemMap<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -263,7 +276,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int q_tile = blockIdx.x;
+  const int q_tiles = (p.tokens + BM - 1) / BM;
+  const int tile0 = 2 * blockIdx.x;                 // this CTA's query tiles: tile0, tile0+1
+  const int n_q = min(2, q_tiles - tile0);          // 1 for an odd last pair
   const int split = blockIdx.y;
   const int head = blockIdx.z;
   const int t_begin = split * p.tiles_per_split;
@@ -276,17 +291,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar = [&](const uint64_t& b) { return smem_u32(&b); };
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(bars->q_full), 1);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(bar(bars->s_full[b]), 1);
-      mbar_init(bar(bars->s_free[b]), 128);
-      mbar_init(bar(bars->p_full[b]), 128);
-      mbar_init(bar(bars->pv_done[b]), 1);
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(bar(bars->q_full[g]), 1);
+      mbar_init(bar(bars->s_full[g]), 1);
+      mbar_init(bar(bars->s_free[g]), 128);
+      mbar_init(bar(bars->p_full[g]), 128);
+      mbar_init(bar(bars->pv_done[g]), 1);
+      mbar_init(bar(bars->drain[g]), 1);
     }
-    mbar_init(bar(bars->drain), 1);
     for (int s = 0; s < C::NS; ++s) {
       mbar_init(bar(bars->kv_full[s]), 1);
-      mbar_init(bar(bars->kv_empty[s]), 1);
+      mbar_init(bar(bars->kv_empty[s]), n_q);
     }
     bars->abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -302,16 +317,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
-
+  if (warp < 4) {
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
       int issued = 0;
-      mbar_expect_tx(bar(bars->q_full), C::TILE_BYTES);
+      for (int g = 0; g < n_q; ++g) {
+        mbar_expect_tx(bar(bars->q_full[g]), C::TILE_BYTES);
 #pragma unroll
-      for (int a = 0; a < C::ATOMS; ++a)
-        tma_load_3d(sQ + a * C::ATOM_BYTES, &p.tm_q, 64 * a, head, q_tile * BM,
-                    bar(bars->q_full));
+        for (int a = 0; a < C::ATOMS; ++a)
+          tma_load_3d(sQ + g * C::TILE_BYTES + a * C::ATOM_BYTES, &p.tm_q, 64 * a, head,
+                      (tile0 + g) * BM, bar(bars->q_full[g]));
+      }
       for (int j = 0; j < n; ++j) {
         const int s = j % C::NS;
         if (j >= C::NS &&
@@ -332,7 +349,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (*abort_flag) {
         // drain: wait (bounded) for the copies this thread issued that may still be landing
-        mbar_wait(bar(bars->q_full), 0, abort_flag, p.err, 0);
+        for (int g = 0; g < n_q; ++g) {
+          const unsigned long long t0 = global_timer();
+          while (!mbar_try(bar(bars->q_full[g]), 0) && global_timer() - t0 < kWaitLimitNs) {
+          }
+        }
         for (int j = max(0, issued - C::NS); j < issued; ++j) {
           const unsigned long long t0 = global_timer();
           while (!mbar_try(bar(bars->kv_full[j % C::NS]), (j / C::NS) & 1) &&
@@ -341,16 +362,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0) {
+  } else if (warp == 1 || warp == 2) {
+    // ---------------- MMA issuers: warp 1 for query tile 0, warp 2 for tile 1 ----------------
+    const int g = warp - 1;
+    if (lane == 0 && g < n_q) {
       constexpr uint32_t idesc_s = idesc_bf16(BM, BN, false);
       constexpr uint32_t idesc_o = idesc_bf16(BM, D, true);
-      bool ok = mbar_wait(bar(bars->q_full), 0, abort_flag, p.err, 2);
+      const uint32_t tS = tmem + 256 * g + TM::S;
+      const uint32_t tP = tmem + 256 * g + TM::P;
+      const uint32_t tO = tmem + 256 * g + TM::O;
+      const uint32_t q_base = sQ + g * C::TILE_BYTES;
+      bool ok = mbar_wait(bar(bars->q_full[g]), 0, abort_flag, p.err, 2);
       tc_fence_after();
+      auto issue_qk = [&](int j) -> bool {
+        const int s = j % C::NS;
+        if (!mbar_wait(bar(bars->kv_full[s]), (j / C::NS) & 1, abort_flag, p.err, 4))
+          return false;
+        if (j >= 1 && !mbar_wait(bar(bars->s_free[g]), (j - 1) & 1, abort_flag, p.err, 5))
+          return false;
+        tc_fence_after();
+        const uint32_t k_base = sK + s * C::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::ATOM_BYTES + (kk & 3) * 32;
+          mma_ss(tS, sdesc(q_base + off, 16, 1024), sdesc(k_base + off, 16, 1024), idesc_s,
+                 kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar(bars->s_full[g]));
+        return true;
+      };
       auto issue_pv = [&](int i) -> bool {
-        const int b = i & 1;
-        if (!mbar_wait(bar(bars->p_full[b]), (i >> 1) & 1, abort_flag, p.err, 3)) return false;
+        if (!mbar_wait(bar(bars->p_full[g]), i & 1, abort_flag, p.err, 3)) return false;
         tc_fence_after();
         const int s = i % C::NS;
         const uint32_t v_base = sV + s * C::TILE_BYTES;
@@ -358,76 +400,74 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < BN / 16; ++kk) {
           // B = V tile [keys][D], MN-major: 16 keys = 2 groups of 8 rows of 128 B
           const uint64_t bd = sdesc(v_base + kk * 2048, C::ATOM_BYTES, 1024);
-          mma_ts(tmem + TM_O, tmem + TM_P + 64 * b + 8 * kk, bd, idesc_o,
-                 (i > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(tO, tP + 8 * kk, bd, idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit(bar(bars->pv_done[b]));
+        mma_commit(bar(bars->pv_done[g]));
         mma_commit(bar(bars->kv_empty[s]));
         return true;
       };
-      for (int j = 0; ok && j < n; ++j) {
-        const int s = j % C::NS;
-        const int b = j & 1;
-        if (!mbar_wait(bar(bars->kv_full[s]), (j / C::NS) & 1, abort_flag, p.err, 4)) break;
-        if (j >= 2 && !mbar_wait(bar(bars->s_free[b]), ((j - 2) >> 1) & 1, abort_flag, p.err, 5))
-          break;
-        tc_fence_after();
-        const uint32_t k_base = sK + s * C::TILE_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::ATOM_BYTES + (kk & 3) * 32;
-          mma_ss(tmem + TM_S + 128 * b, sdesc(sQ + off, 16, 1024), sdesc(k_base + off, 16, 1024),
-                 idesc_s, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(bar(bars->s_full[b]));
-        if (j >= 1 && !issue_pv(j - 1)) {
-          ok = false;
-          break;
+      if (ok && n > 0) ok = issue_qk(0);
+      for (int j = 1; ok && j < n; ++j) {
+        if (TM::kPAliasesS) {
+          // P_{j-1} lives in S: PV_{j-1} must have read it before S_j overwrites it
+          ok = issue_pv(j - 1) &&
+               mbar_wait(bar(bars->pv_done[g]), (j - 1) & 1, abort_flag, p.err, 10) &&
+               issue_qk(j);
+        } else {
+          // S_j only needs S_{j-1} read: issue it first so the softmax can start early
+          ok = issue_qk(j) && issue_pv(j - 1);
         }
       }
       if (ok && !*abort_flag && n > 0) issue_pv(n - 1);
       // every MMA issued by this thread has completed once `drain` flips
-      mma_commit(bar(bars->drain));
+      mma_commit(bar(bars->drain[g]));
       const unsigned long long t0 = global_timer();
-      while (!mbar_try(bar(bars->drain), 0) && global_timer() - t0 < kWaitLimitNs) {
+      while (!mbar_try(bar(bars->drain[g]), 0) && global_timer() - t0 < kWaitLimitNs) {
       }
     }
+  }
   } else {
-    // ---------------- softmax + epilogue (warps 2..5) ----------------
+    // ---------------- softmax + epilogue: warps 4..7 tile 0, warps 8..11 tile 1 ----------------
+    const int g = (warp - 4) >> 2;
     const int quad = warp & 3;                  // TMEM lane quadrant this warp may access
-    const int row_in_tile = quad * 32 + lane;
-    const int row = q_tile * BM + row_in_tile;
-    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+    const int row = (tile0 + g) * BM + quad * 32 + lane;
+    const uint32_t lane_base = tmem + 256 * g + ((uint32_t)(quad * 32) << 16);
+    const uint32_t tS = lane_base + TM::S;
+    const uint32_t tP = lane_base + TM::P;
+    const uint32_t tO = lane_base + TM::O;
     float m = -INFINITY;  // running max (log2 domain) the P values and O are relative to
     float l = 0.f;
-    bool ok = true;
+    bool ok = g < n_q;
     uint32_t S[BN];
-    for (int j = 0; j < n; ++j) {
-      const int b = j & 1;
+    for (int j = 0; ok && j < n; ++j) {
       // every wait in these warps is made warp-uniform, so warp-collective tcgen05 ops and
       // votes below always run with the whole warp
-      if (!__all_sync(kFull, mbar_wait(bar(bars->s_full[b]), (j >> 1) & 1, abort_flag, p.err, 6))) {
+      if (!__all_sync(kFull, mbar_wait(bar(bars->s_full[g]), j & 1, abort_flag, p.err, 6))) {
         ok = false;
         break;
       }
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < BN / 32; ++c) tmem_ld32(lane_base + TM_S + 128 * b + 32 * c, S + 32 * c);
+      for (int c = 0; c < BN / 32; ++c) tmem_ld32(tS + 32 * c, S + 32 * c);
       tmem_wait_ld();
       reg_fence<BN>(S);
       tc_fence_before();
-      mbar_arrive(bar(bars->s_free[b]));
+      mbar_arrive(bar(bars->s_free[g]));
 
       const int valid = tile_ref(p, t_begin + j).valid;
-      float mx = -INFINITY;
+      float mx8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
       if (valid == BN) {
 #pragma unroll
-        for (int i = 0; i < BN; ++i) mx = fmaxf(mx, __uint_as_float(S[i]));
+        for (int i = 0; i < BN; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], __uint_as_float(S[i]));
       } else {
 #pragma unroll
         for (int i = 0; i < BN; ++i)
-          if (i < valid) mx = fmaxf(mx, __uint_as_float(S[i]));
+          if (i < valid) mx8[i & 7] = fmaxf(mx8[i & 7], __uint_as_float(S[i]));
       }
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float m_tile = mx * p.scale_log2;
       bool rescale = false;
       float alpha = 1.f;
@@ -437,13 +477,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         l *= alpha;
         rescale = true;
       }
-      // P_j goes to P[b]: PV_{j-2} must have finished reading it
-      if (j >= 2 && !__all_sync(kFull, mbar_wait(bar(bars->pv_done[b]), ((j - 2) >> 1) & 1,
+      // P_j overwrites P_{j-1} (and O may be rescaled): PV_{j-1} must have finished
+      if (j >= 1 && !__all_sync(kFull, mbar_wait(bar(bars->pv_done[g]), (j - 1) & 1,
                                                  abort_flag, p.err, 7))) {
         ok = false;
         break;
       }
+      tc_fence_after();
       const float neg_m = -m;
+      float l8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) l8[i] = 0.f;
 #pragma unroll
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t pk[16];
@@ -456,38 +500,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (i0 >= valid) p0 = 0.f;
             if (i0 + 1 >= valid) p1 = 0.f;
           }
-          l += p0 + p1;
+          l8[i & 7] += p0 + p1;
           pk[i] = pack_bf16(p0, p1);
         }
-        tmem_st16(lane_base + TM_P + 64 * b + 16 * c, pk);
+        tmem_st16(tP + 16 * c, pk);
       }
-      if (__any_sync(0xffffffffu, rescale) && j > 0) {
+      l += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
+      if (__any_sync(kFull, rescale) && j > 0) {
         // O holds sum_{i<j} P_i V_i relative to the old max: scale it before PV_j lands
-        if (!__all_sync(kFull, mbar_wait(bar(bars->pv_done[(j - 1) & 1]), ((j - 1) >> 1) & 1,
-                                         abort_flag, p.err, 8))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
-          tmem_ld32(lane_base + TM_O + 32 * c, o);
+          tmem_ld32(tO + 32 * c, o);
           tmem_wait_ld();
           reg_fence<32>(o);
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st16(lane_base + TM_O + 32 * c, o);
-          tmem_st16(lane_base + TM_O + 32 * c + 16, o + 16);
+          tmem_st16(tO + 32 * c, o);
+          tmem_st16(tO + 32 * c + 16, o + 16);
         }
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(bars->p_full[b]));
+      mbar_arrive(bar(bars->p_full[g]));
     }
     if (ok && n > 0 &&
-        __all_sync(kFull, mbar_wait(bar(bars->pv_done[(n - 1) & 1]), ((n - 1) >> 1) & 1,
-                                    abort_flag, p.err, 9))) {
+        __all_sync(kFull, mbar_wait(bar(bars->pv_done[g]), (n - 1) & 1, abort_flag, p.err, 9))) {
       tc_fence_after();
       const float inv_l = 1.f / l;
       const bool store = row < p.tokens;
@@ -497,7 +535,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
-          tmem_ld32(lane_base + TM_O + 32 * c, o);
+          tmem_ld32(tO + 32 * c, o);
           tmem_wait_ld();
           reg_fence<32>(o);
           if (store) {
@@ -518,7 +556,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
-          tmem_ld32(lane_base + TM_O + 32 * c, o);
+          tmem_ld32(tO + 32 * c, o);
           tmem_wait_ld();
           reg_fence<32>(o);
           if (store) {
@@ -581,26 +619,27 @@ size_t attn_tc_smem_bytes(int head_dim) {
   return head_dim == 64 ? Cfg<64>::SMEM : Cfg<128>::SMEM;
 }
 
+namespace {
+
+template <int D>
+cudaError_t prepare_attn_tc() {
+  static cudaError_t state = cudaErrorNotReady;
+  if (state == cudaErrorNotReady)
+    state = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Cfg<D>::SMEM);
+  return state;
+}
+
+}  // namespace
+
 cudaError_t launch_attn_tc(const AttnParams& p, int head_dim, int q_tiles, cudaStream_t s) {
-  dim3 grid(q_tiles, p.n_splits, p.heads);
+  dim3 grid((q_tiles + 1) / 2, p.n_splits, p.heads);
   cudaError_t e;
   if (head_dim == 64) {
-    static bool attr = false;
-    if (!attr) {
-      e = cudaFuncSetAttribute(attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               Cfg<64>::SMEM);
-      if (e != cudaSuccess) return e;
-      attr = true;
-    }
+    if ((e = prepare_attn_tc<64>()) != cudaSuccess) return e;
     attn_tc_kernel<64><<<grid, kThreads, Cfg<64>::SMEM, s>>>(p);
   } else if (head_dim == 128) {
-    static bool attr = false;
-    if (!attr) {
-      e = cudaFuncSetAttribute(attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               Cfg<128>::SMEM);
-      if (e != cudaSuccess) return e;
-      attr = true;
-    }
+    if ((e = prepare_attn_tc<128>()) != cudaSuccess) return e;
     attn_tc_kernel<128><<<grid, kThreads, Cfg<128>::SMEM, s>>>(p);
   } else {
     return cudaErrorInvalidValue;

@@ -375,7 +375,8 @@ int lbm_attend_frame(lbm_cache_t* c, const void* q, void* out, void* stream) {
     for (size_t i = 0; i < pages.size(); ++i) p.pages[i] = (uint16_t)pages[i];
     const int q_tiles = (T + 127) / 128;
     const double combine = (double)T * c->heads * c->head_dim * 4.0 / 1.8e6;
-    p.n_splits = plan_splits(q_tiles * c->heads, p.n_tiles, c->num_sms, combine, c->max_splits);
+    p.n_splits = plan_splits((q_tiles + 1) / 2 * c->heads, p.n_tiles, c->num_sms, combine,
+                             c->max_splits);
     if (c->forced_splits) p.n_splits = std::min(c->forced_splits, p.n_tiles);
     p.tiles_per_split = (p.n_tiles + p.n_splits - 1) / p.n_splits;
     p.n_splits = (p.n_tiles + p.tiles_per_split - 1) / p.tiles_per_split;  // no empty split
