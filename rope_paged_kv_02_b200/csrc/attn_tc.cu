@@ -41,6 +41,9 @@ constexpr uint32_t kTmemCols = 512;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when max grows by > 2^8
 constexpr unsigned kFull = 0xffffffffu;
+// a waiting thread may sleep in mbarrier.try_wait up to this long before re-checking the
+// time limit, instead of spinning and taking issue slots from the softmax warps
+constexpr uint32_t kSuspendHintNs = 1000000;
 
 template <int D>
 struct Cfg {
@@ -79,10 +82,10 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
       : "memory");
   return ok != 0;
 }
@@ -212,6 +215,35 @@ __device__ __forceinline__ float fast_exp2(float x) {
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&b);
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+__device__ __forceinline__ uint64_t pack_f2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+
+__device__ __forceinline__ void unpack_f2(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+
+// (a0, a1) * (b, b) + (c, c) on the paired fp32 pipe
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.ftz.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.ftz.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
 }
 
 // Key tile t of the visible list: pool (patch or special), first pool row, valid keys.
@@ -455,19 +487,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(bar(bars->s_free[g]));
 
       const int valid = tile_ref(p, t_begin + j).valid;
-      float mx8[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
-      if (valid == BN) {
-#pragma unroll
-        for (int i = 0; i < BN; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], __uint_as_float(S[i]));
-      } else {
+      if (valid != BN) {
+        // keys past the end of a page / of the special stream: -inf scores, zero weight
 #pragma unroll
         for (int i = 0; i < BN; ++i)
-          if (i < valid) mx8[i & 7] = fmaxf(mx8[i & 7], __uint_as_float(S[i]));
+          if (i >= valid) S[i] = 0xff800000u;
       }
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      float mx8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        mx8[i] = fmaxf(__uint_as_float(S[2 * i]), __uint_as_float(S[2 * i + 1]));
+#pragma unroll
+      for (int i = 16; i < BN; i += 2)
+        mx8[(i >> 1) & 7] = max3f(mx8[(i >> 1) & 7], __uint_as_float(S[i]),
+                                  __uint_as_float(S[i + 1]));
+      const float mx = max3f(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]),
+                             fmaxf(mx8[6], mx8[7]));
       const float m_tile = mx * p.scale_log2;
       bool rescale = false;
       float alpha = 1.f;
@@ -484,28 +519,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const float neg_m = -m;
-      float l8[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) l8[i] = 0.f;
+      const uint64_t c2 = pack_f2(p.scale_log2, p.scale_log2);
+      const uint64_t nm2 = pack_f2(-m, -m);
+      uint64_t l4[4] = {0, 0, 0, 0};
 #pragma unroll
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int i0 = 32 * c + 2 * i;
-          float p0 = fast_exp2(fmaf(__uint_as_float(S[i0]), p.scale_log2, neg_m));
-          float p1 = fast_exp2(fmaf(__uint_as_float(S[i0 + 1]), p.scale_log2, neg_m));
-          if (valid != BN) {
-            if (i0 >= valid) p0 = 0.f;
-            if (i0 + 1 >= valid) p1 = 0.f;
-          }
-          l8[i & 7] += p0 + p1;
+          float x0, x1;
+          unpack_f2(ffma2(pack_f2(__uint_as_float(S[i0]), __uint_as_float(S[i0 + 1])), c2, nm2),
+                    x0, x1);
+          const float p0 = fast_exp2(x0);
+          const float p1 = fast_exp2(x1);
+          l4[i & 3] = fadd2(l4[i & 3], pack_f2(p0, p1));
           pk[i] = pack_bf16(p0, p1);
         }
         tmem_st16(tP + 16 * c, pk);
       }
-      l += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
+      {
+        float a0, a1, b0, b1, c0, c1, d0, d1;
+        unpack_f2(l4[0], a0, a1);
+        unpack_f2(l4[1], b0, b1);
+        unpack_f2(l4[2], c0, c1);
+        unpack_f2(l4[3], d0, d1);
+        l += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
+      }
       if (__any_sync(kFull, rescale) && j > 0) {
         // O holds sum_{i<j} P_i V_i relative to the old max: scale it before PV_j lands
 #pragma unroll

@@ -100,67 +100,67 @@ __device__ __forceinline__ U4 rotate_chunk<float>(const RopeTables& rt, U4 in, i
 constexpr int kAppendThreads = 256;
 constexpr int kAppendUnroll = 4;
 
-// Grid-stride over 3 * T * H * (D / EPC) chunks: tensor-major (q, k, v), then token,
-// head, chunk, so neighbouring threads touch neighbouring 16-byte chunks.
-template <typename T>
+// One pass over the 3 * T * H * (D / EPC) 16-byte chunks of q, k, v (32-bit indices: a
+// frame is far below 2^31 chunks): tensor-major (q, k, v), then token, head, chunk, so
+// neighbouring threads touch neighbouring 16-byte chunks.  CPR = chunks per (token, head)
+// row is a compile-time power of two, so only the division by the head count is a real one.
+template <typename T, int CPR>
 __global__ void __launch_bounds__(kAppendThreads)
     rope_append_kernel(RopeTables rt, Pools pools, AppendArgs a) {
   constexpr int EPC = 16 / sizeof(T);
-  const int cpr = a.head_dim / EPC;                 // chunks per (token, head) row
-  const long long per_tensor = (long long)a.tokens * a.heads * cpr;
-  const long long total = 3 * per_tensor;
-  const int ppw = rt.ppw;
-  const long long stride_all = (long long)gridDim.x * blockDim.x * kAppendUnroll;
-  for (long long base = (long long)blockIdx.x * blockDim.x * kAppendUnroll + threadIdx.x;
-       base < total; base += stride_all) {
+  const uint32_t per_tensor = (uint32_t)a.tokens * a.heads * CPR;
+  const uint32_t total = 3u * per_tensor;
+  const uint32_t stride_all = gridDim.x * blockDim.x * kAppendUnroll;
+  for (uint32_t base = blockIdx.x * blockDim.x * kAppendUnroll + threadIdx.x; base < total;
+       base += stride_all) {
     U4 val[kAppendUnroll];
     // issue every load of this round before any arithmetic (memory-level parallelism)
 #pragma unroll
     for (int u = 0; u < kAppendUnroll; ++u) {
-      const long long idx = base + (long long)u * blockDim.x;
+      const uint32_t idx = base + u * blockDim.x;
       if (idx < total) {
-        const int tensor = (int)(idx / per_tensor);
-        const long long rem = idx - tensor * per_tensor;
+        const uint32_t tensor = idx >= per_tensor ? (idx >= 2 * per_tensor ? 2u : 1u) : 0u;
+        const uint32_t rem = idx - tensor * per_tensor;
         const char* src = tensor == 0 ? (const char*)a.q : tensor == 1 ? (const char*)a.k
                                                                        : (const char*)a.v;
-        src += rem * 16;
+        src += (size_t)rem * 16;
         val[u] = tensor == 0 ? ld_plain(src) : ld_stream(src);
       }
     }
 #pragma unroll
     for (int u = 0; u < kAppendUnroll; ++u) {
-      const long long idx = base + (long long)u * blockDim.x;
+      const uint32_t idx = base + u * blockDim.x;
       if (idx >= total) continue;
-      const int tensor = (int)(idx / per_tensor);
-      const long long rem = idx - tensor * per_tensor;
-      const int c = (int)(rem % cpr);
-      const long long th = rem / cpr;
-      const int h = (int)(th % a.heads);
-      const int j = (int)(th / a.heads);
+      const uint32_t tensor = idx >= per_tensor ? (idx >= 2 * per_tensor ? 2u : 1u) : 0u;
+      const uint32_t rem = idx - tensor * per_tensor;
+      const int c = (int)(rem % CPR);
+      const uint32_t th = rem / CPR;
+      const int j = (int)(th / (uint32_t)a.heads);
+      const int h = (int)(th - (uint32_t)j * a.heads);
       const int d0 = c * EPC;
       U4 out = val[u];
       if (tensor < 2) {
         int hh = 0, ww = 0;
         if (j >= a.psi) {
           const int pj = j - a.psi;
-          hh = 1 + pj / ppw;
-          ww = 1 + pj % ppw;
+          hh = 1 + pj / rt.ppw;
+          ww = 1 + pj - (hh - 1) * rt.ppw;
         }
         out = rotate_chunk<T>(rt, out, d0, a.frame, hh, ww);
       }
       char* dst;
       if (tensor == 0) {
-        dst = (char*)a.q + rem * 16;
+        dst = (char*)a.q + (size_t)rem * 16;
       } else {
         const bool special = j < a.psi;
         void* pool = special ? (tensor == 1 ? pools.k_special : pools.v_special)
                              : (tensor == 1 ? pools.k_patch : pools.v_patch);
-        long long row;
+        size_t row;
         if (special)
-          row = (long long)h * pools.spec_cap + a.special_slot + j;
+          row = (size_t)h * pools.spec_cap + a.special_slot + j;
         else
-          row = ((long long)h * pools.num_pages + a.page) * pools.page_stride + (j - a.psi);
-        dst = (char*)pool + (row * a.head_dim + d0) * (long long)sizeof(T);
+          row = ((size_t)h * pools.num_pages + a.page) * pools.page_stride + (j - a.psi);
+        dst = (char*)pool + (row * CPR + c) * 16;
       }
       st_plain(dst, out);
     }
@@ -203,15 +203,24 @@ cudaError_t launch_rope_expand(const RopeTables& rt, float* cos_out, float* sin_
 cudaError_t launch_rope_append(const RopeTables& rt, const Pools& pools, const AppendArgs& a,
                                cudaStream_t s) {
   const int esz = a.dtype == LBM_BF16 ? 2 : 4;
-  const long long chunks = 3LL * a.tokens * a.heads * (a.head_dim * esz / 16);
+  const int cpr = a.head_dim * esz / 16;
+  const long long chunks = 3LL * a.tokens * a.heads * cpr;
+  if (chunks >= (1LL << 31)) return cudaErrorInvalidValue;
   const long long per_block = (long long)kAppendThreads * kAppendUnroll;
   long long blocks = (chunks + per_block - 1) / per_block;
   if (blocks > 148 * 8) blocks = 148 * 8;
   if (blocks < 1) blocks = 1;
-  if (a.dtype == LBM_BF16)
-    rope_append_kernel<__nv_bfloat16><<<(unsigned)blocks, kAppendThreads, 0, s>>>(rt, pools, a);
+  const dim3 grid((unsigned)blocks);
+  if (a.dtype == LBM_BF16 && cpr == 8)
+    rope_append_kernel<__nv_bfloat16, 8><<<grid, kAppendThreads, 0, s>>>(rt, pools, a);
+  else if (a.dtype == LBM_BF16 && cpr == 16)
+    rope_append_kernel<__nv_bfloat16, 16><<<grid, kAppendThreads, 0, s>>>(rt, pools, a);
+  else if (a.dtype == LBM_F32 && cpr == 16)
+    rope_append_kernel<float, 16><<<grid, kAppendThreads, 0, s>>>(rt, pools, a);
+  else if (a.dtype == LBM_F32 && cpr == 32)
+    rope_append_kernel<float, 32><<<grid, kAppendThreads, 0, s>>>(rt, pools, a);
   else
-    rope_append_kernel<float><<<(unsigned)blocks, kAppendThreads, 0, s>>>(rt, pools, a);
+    return cudaErrorInvalidValue;
   return cudaGetLastError();
 }
 
