@@ -41,13 +41,17 @@ __device__ __forceinline__ void st_plain(void* p, const U4& r) {
                : "memory");
 }
 
-// (cos, sin) of feature pair i for a token at (t, hh, ww).
+// (cos, sin) of feature pair i for a token at (t, hh, ww): pairs [0, nt) use the t table,
+// [nt, nt+nh) the h table, the rest the w table.  Branch-free (one load), because the lanes
+// of a warp cover different pairs of the same token.
 __device__ __forceinline__ float2 pair_cs(const RopeTables& rt, int i, int t, int hh, int ww) {
-  if (i < rt.nt) return __ldg(rt.tab_t + t * rt.nt + i);
-  i -= rt.nt;
-  if (i < rt.nh) return __ldg(rt.tab_h + hh * rt.nh + i);
-  i -= rt.nh;
-  return __ldg(rt.tab_w + ww * rt.nw + i);
+  const bool in_t = i < rt.nt;
+  const bool in_h = !in_t && i < rt.nt + rt.nh;
+  const float2* base = in_t ? rt.tab_t : (in_h ? rt.tab_h : rt.tab_w);
+  const int pairs = in_t ? rt.nt : (in_h ? rt.nh : rt.nw);
+  const int row = in_t ? t : (in_h ? hh : ww);
+  const int col = in_t ? i : (in_h ? i - rt.nt : i - rt.nt - rt.nh);
+  return __ldg(base + row * pairs + col);
 }
 
 __device__ __forceinline__ void rot(float& x0, float& x1, float2 cs) {
@@ -98,7 +102,7 @@ __device__ __forceinline__ U4 rotate_chunk<float>(const RopeTables& rt, U4 in, i
 }
 
 constexpr int kAppendThreads = 256;
-constexpr int kAppendUnroll = 4;
+constexpr int kAppendUnroll = 1;
 
 // One pass over the 3 * T * H * (D / EPC) 16-byte chunks of q, k, v (32-bit indices: a
 // frame is far below 2^31 chunks): tensor-major (q, k, v), then token, head, chunk, so
@@ -208,7 +212,7 @@ cudaError_t launch_rope_append(const RopeTables& rt, const Pools& pools, const A
   if (chunks >= (1LL << 31)) return cudaErrorInvalidValue;
   const long long per_block = (long long)kAppendThreads * kAppendUnroll;
   long long blocks = (chunks + per_block - 1) / per_block;
-  if (blocks > 148 * 8) blocks = 148 * 8;
+  if (blocks > 148 * 64) blocks = 148 * 64;
   if (blocks < 1) blocks = 1;
   const dim3 grid((unsigned)blocks);
   if (a.dtype == LBM_BF16 && cpr == 8)
