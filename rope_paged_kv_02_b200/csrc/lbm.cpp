@@ -50,6 +50,7 @@ struct lbm_cache {
 namespace {
 
 constexpr int kMaxSplits = 16;
+constexpr int kKeyTile = 64;  // keys per attention key tile (page strides are multiples)
 
 int elem_size(int dtype) { return dtype == LBM_BF16 ? 2 : 4; }
 
@@ -114,7 +115,7 @@ int plan_splits(int work_units, int n_tiles, int num_sms, double combine_tiles_p
     if (s_eff != s) continue;
     const long long units = (long long)work_units * s;
     const long long waves = (units + num_sms - 1) / num_sms;
-    double cost = (double)waves * (tps + 6.0);
+    double cost = (double)waves * (tps + 8.0);
     if (s > 1) cost += 8.0 + combine_tiles_per_split * s;
     if (cost < best_cost - 1e-9) {
       best_cost = cost;
@@ -247,7 +248,7 @@ int lbm_cache_create(int heads, int head_dim, int patches_per_frame, int special
   }
 
   const int P = scale_frames + sliding_window + 1;
-  const int stride = (patches_per_frame + 127) / 128 * 128;
+  const int stride = (patches_per_frame + kKeyTile - 1) / kKeyTile * kKeyTile;
   const long long cap = (6LL * (max_frames + 1) + 127) / 128 * 128;
   const int e = elem_size(dtype);
   const size_t patch_bytes = (size_t)heads * P * stride * head_dim * e;
@@ -292,10 +293,11 @@ int lbm_cache_create(int heads, int head_dim, int patches_per_frame, int special
   if (dtype == LBM_BF16) {
     const uint64_t row = (uint64_t)head_dim * 2;
     const uint64_t prow = (uint64_t)P * stride;
-    if (!make_map(&c->tm_kp, c->pools.k_patch, head_dim, prow, heads, row, prow * row, 128, 1) ||
-        !make_map(&c->tm_vp, c->pools.v_patch, head_dim, prow, heads, row, prow * row, 128, 1) ||
-        !make_map(&c->tm_ks, c->pools.k_special, head_dim, cap, heads, row, cap * row, 128, 1) ||
-        !make_map(&c->tm_vs, c->pools.v_special, head_dim, cap, heads, row, cap * row, 128, 1))
+    const uint32_t kt = kKeyTile;
+    if (!make_map(&c->tm_kp, c->pools.k_patch, head_dim, prow, heads, row, prow * row, kt, 1) ||
+        !make_map(&c->tm_vp, c->pools.v_patch, head_dim, prow, heads, row, prow * row, kt, 1) ||
+        !make_map(&c->tm_ks, c->pools.k_special, head_dim, cap, heads, row, cap * row, kt, 1) ||
+        !make_map(&c->tm_vs, c->pools.v_special, head_dim, cap, heads, row, cap * row, kt, 1))
       return fail(LBM_ERR_CUDA);
   }
   if (cudaDeviceSynchronize() != cudaSuccess) return fail(LBM_ERR_CUDA);
@@ -367,14 +369,15 @@ int lbm_attend_frame(lbm_cache_t* c, const void* q, void* out, void* stream) {
     p.heads = c->heads;
     p.patches = c->patches;
     p.page_stride = c->pools.page_stride;
-    p.tiles_per_page = c->pools.page_stride / 128;
+    p.tiles_per_page = (c->patches + kKeyTile - 1) / kKeyTile;
     p.n_pages = (int)pages.size();
     p.n_special = n_sp;
-    p.n_tiles = p.n_pages * p.tiles_per_page + (n_sp + 127) / 128;
+    p.n_tiles = p.n_pages * p.tiles_per_page + (n_sp + kKeyTile - 1) / kKeyTile;
     p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)c->head_dim));
     for (size_t i = 0; i < pages.size(); ++i) p.pages[i] = (uint16_t)pages[i];
     const int q_tiles = (T + 127) / 128;
-    const double combine = (double)T * c->heads * c->head_dim * 4.0 / 1.8e6;
+    // combine cost of one split, in key-tile times (a tile of both query tiles ~0.5 us)
+    const double combine = (double)T * c->heads * c->head_dim * 4.0 / 3.0e6;
     p.n_splits = plan_splits((q_tiles + 1) / 2 * c->heads, p.n_tiles, c->num_sms, combine,
                              c->max_splits);
     if (c->forced_splits) p.n_splits = std::min(c->forced_splits, p.n_tiles);
