@@ -9,7 +9,7 @@
 // (64 keys each).  Both query tiles share every K/V tile the CTA loads.  Warp roles:
 //   warp 0      TMA producer: the two Q tiles once, then K/V tiles gathered page by page
 //               through the page table into a ring of shared-memory stages (128B swizzle).
-//   warp 1, 2   allocate tensor memory (warp 1); one lane of warp 1+g issues every
+//   warp 1, 2   allocate tensor memory (warp 1); warp 1+g issues (one elected lane) every
 //               tcgen05.mma of query tile g:
 //                 S_j = Q_g K_j^T  (A, B from shared memory)      -> TMEM S buffer j % 2
 //                 O_g += P_j V_j   (A = P from TMEM, B = V smem)   -> TMEM O_g
@@ -68,9 +68,15 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
 
+// The issue helpers below (expect_tx, TMA, MMA, commit) are called by a whole warp in
+// warp-uniform control flow; one elected lane issues the instruction.  Keeping the loop
+// warp-uniform lets the compiler hold descriptors and addresses in uniform registers.
 __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-               : "memory");
+  asm volatile(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n\t}" ::"r"(bar),
+      "r"(bytes)
+      : "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
@@ -115,8 +121,9 @@ __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile i
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* tm, int x, int y,
                                             int z, uint32_t bar) {
   asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];\n\t}" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(z), "r"(bar)
       : "memory");
 }
@@ -143,9 +150,10 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major)
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                        uint32_t idesc, uint32_t accum) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred p, e;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accum)
       : "memory");
 }
@@ -153,16 +161,19 @@ __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_
 __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                        uint32_t idesc, uint32_t accum) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred p, e;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accum)
       : "memory");
 }
 
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}"
+      ::"r"(bar)
       : "memory");
 }
 
@@ -352,8 +363,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = bars->tmem_base;
 
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
-    if (lane == 0) {
+    // ---------------- TMA producer (whole warp, elected lane issues) ----------------
+    {
       int issued = 0;
       for (int g = 0; g < n_q; ++g) {
         mbar_expect_tx(bar(bars->q_full[g]), C::Q_BYTES);
@@ -364,8 +375,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int j = 0; j < n; ++j) {
         const int s = j % C::NS;
-        if (j >= C::NS &&
-            !mbar_wait(bar(bars->kv_empty[s]), ((j - C::NS) / C::NS) & 1, abort_flag, p.err, 1))
+        if (j >= C::NS && !__all_sync(kFull, mbar_wait(bar(bars->kv_empty[s]),
+                                                       ((j - C::NS) / C::NS) & 1, abort_flag,
+                                                       p.err, 1)))
           break;
         const TileRef t = tile_ref(p, t_begin + j);
         const CUtensorMap* tk = t.special ? &p.tm_ks : &p.tm_kp;
@@ -398,22 +410,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1 || warp == 2) {
     // ---------------- MMA issuers: warp 1 for query tile 0, warp 2 for tile 1 ----------------
     const int g = warp - 1;
-    if (lane == 0 && g < n_q) {
+    if (g < n_q) {  // whole warp, elected lane issues
       constexpr uint32_t idesc_s = idesc_bf16(BM, BN, false);
       constexpr uint32_t idesc_o = idesc_bf16(BM, D, true);
       const uint32_t tG = tmem + 256 * g;
       const uint32_t q_base = sQ + g * C::Q_BYTES;
-      bool ok = mbar_wait(bar(bars->q_full[g]), 0, abort_flag, p.err, 2);
+      bool ok = __all_sync(kFull, mbar_wait(bar(bars->q_full[g]), 0, abort_flag, p.err, 2));
       tc_fence_after();
       auto issue_qk = [&](int j) -> bool {
         const int s = j % C::NS;
         const int b = j & 1;
-        if (!mbar_wait(bar(bars->kv_full[s]), (j / C::NS) & 1, abort_flag, p.err, 4))
+        if (!__all_sync(kFull, mbar_wait(bar(bars->kv_full[s]), (j / C::NS) & 1, abort_flag, p.err, 4)))
           return false;
         // S buffer b held S_{j-2} (and, with head_dim 128, P_{j-2}): wait until it is free
-        if (j >= 2 && !mbar_wait(TM::kPAliasesS ? bar(bars->pv_done[g][b])
-                                                : bar(bars->s_free[g][b]),
-                                 ((j - 2) >> 1) & 1, abort_flag, p.err, 5))
+        if (j >= 2 && !__all_sync(kFull, mbar_wait(TM::kPAliasesS ? bar(bars->pv_done[g][b])
+                                                                  : bar(bars->s_free[g][b]),
+                                                   ((j - 2) >> 1) & 1, abort_flag, p.err, 5)))
           return false;
         tc_fence_after();
         const uint32_t k_base = sK + s * C::KV_BYTES;
@@ -429,7 +441,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       auto issue_pv = [&](int i) -> bool {
         const int b = i & 1;
-        if (!mbar_wait(bar(bars->p_full[g][b]), (i >> 1) & 1, abort_flag, p.err, 3)) return false;
+        if (!__all_sync(kFull, mbar_wait(bar(bars->p_full[g][b]), (i >> 1) & 1, abort_flag,
+                                         p.err, 3)))
+          return false;
         tc_fence_after();
         const int s = i % C::NS;
         const uint32_t v_base = sV + s * C::KV_BYTES;
