@@ -109,7 +109,7 @@ LBM_API void lbm_rope_destroy(lbm_rope_t* rope);
  *   dtype              LBM_BF16 (tensor-core path) or LBM_F32 (exact SIMT path)
  *   rope               tables built for the same head_dim / grid; must outlive the cache
  * Device memory: K and V patch pools [heads][P*stride][head_dim] with P = scale_frames +
- * sliding_window + 1 pages and stride = patches_per_frame rounded up to 64 (zero-filled);
+ * sliding_window + 1 pages and stride = patches_per_frame rounded up to 128 (zero-filled);
  * K and V special pools [heads][cap][head_dim], cap = 6*(max_frames+1) rounded up to 128;
  * split-KV scratch.  Synchronous. */
 LBM_API int lbm_cache_create(int heads, int head_dim, int patches_per_frame, int specials_per_frame,

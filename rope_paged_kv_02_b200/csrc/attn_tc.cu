@@ -5,21 +5,24 @@
 // over the visible page table (scale pages -> window pages -> own page -> special pages,
 // the last special page partly filled), with K/V that already carry their rotation.
 //
-// One CTA = two query tiles of 128 rows of one head, over one split of the key tiles
-// (64 keys each).  Both query tiles share every K/V tile the CTA loads.  Warp roles:
+// One CTA = two query tiles of 128 rows of one head, over one split of the key tiles.
+// Both query tiles share every K/V tile the CTA loads.  Warp roles (12 warps):
 //   warp 0      TMA producer: the two Q tiles once, then K/V tiles gathered page by page
 //               through the page table into a ring of shared-memory stages (128B swizzle).
-//   warp 1, 2   allocate tensor memory (warp 1); warp 1+g issues (one elected lane) every
+//   warp 1, 2   allocate tensor memory (warp 1); one lane of warp 1+g issues every
 //               tcgen05.mma of query tile g:
-//                 S_j = Q_g K_j^T  (A, B from shared memory)      -> TMEM S buffer j % 2
-//                 O_g += P_j V_j   (A = P from TMEM, B = V smem)   -> TMEM O_g
-//               S and P are double-buffered, so the tensor core computes S_{j+2} / PV_j
-//               while the softmax warps work on tile j+1.
+//                 S = Q_g K_j^T   (A, B from shared memory)      -> TMEM S_g
+//                 O_g += P V_j    (A = P from TMEM, B = V smem)   -> TMEM O_g
+//               With head_dim 64, S_{j+1} is issued as soon as the softmax warps have read
+//               S_j, before PV_j, so scores and softmax overlap.
 //   warps 4..7  softmax of query tile 0, warps 8..11 of tile 1: each thread owns one query
 //               row (its TMEM lane); reads S_j, row max, exp2, row sum in fp32, writes P_j
 //               (bf16) into TMEM, and rescales O only when the running max grew by more than
 //               2^8 (lazy rescale; exact because O and l share one reference max).
-// Tensor memory: 256 columns per query tile (layout in TmemMap).
+//   The two softmax warpgroups run concurrently, so one's exponentials overlap the other's
+//   tensor-core work.
+// Tensor memory: 256 columns per query tile g at 256 g: S [0,128); head_dim 64:
+// P [128,192), O [192,256); head_dim 128: O [128,256), P written over S [0,64).
 // Every mbarrier wait is bounded (about 2 s); a wait that runs out sets the device error
 // word, raises a CTA-wide abort flag, and every role falls through to the common exit,
 // which drains outstanding copies / MMAs (bounded) and frees tensor memory.
@@ -31,8 +34,8 @@
 namespace lbm {
 namespace {
 
-constexpr int BM = 128;         // query rows per query tile
-constexpr int BN = 64;          // keys per key tile
+constexpr int BM = 128;         // query rows per CTA
+constexpr int BN = 128;         // keys per tile
 constexpr int kThreads = 384;   // 12 warps
 constexpr uint32_t kTmemCols = 512;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
@@ -44,17 +47,15 @@ constexpr uint32_t kSuspendHintNs = 1000000;
 
 template <int D>
 struct Cfg {
-  static constexpr int ATOMS = D / 64;              // 128-byte swizzle atoms along head_dim
-  static constexpr int Q_ATOM = BM * 128;           // one atom of a query tile
-  static constexpr int KV_ATOM = BN * 128;          // one atom of a key or value tile
-  static constexpr int Q_BYTES = ATOMS * Q_ATOM;
-  static constexpr int KV_BYTES = ATOMS * KV_ATOM;
-  static constexpr int NS = D == 64 ? 8 : 4;        // K/V ring stages
-  static constexpr int OFF_Q = 0;                   // two query tiles
-  static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
-  static constexpr int OFF_V = OFF_K + NS * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_V + NS * KV_BYTES;
-  static constexpr int BAR_BYTES = 512;
+  static constexpr int NS = D == 64 ? 4 : 2;            // K/V pipeline stages
+  static constexpr int ATOM_BYTES = 128 * 128;          // 128 rows x 64 bf16 (one swizzle atom column)
+  static constexpr int ATOMS = D / 64;
+  static constexpr int TILE_BYTES = ATOMS * ATOM_BYTES; // one Q, K or V tile
+  static constexpr int OFF_Q = 0;                       // two query tiles
+  static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
+  static constexpr int OFF_V = OFF_K + NS * TILE_BYTES;
+  static constexpr int OFF_BAR = OFF_V + NS * TILE_BYTES;
+  static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM = OFF_BAR + BAR_BYTES + 1024;  // + slack to align the base to 1 KB
 };
 
@@ -103,9 +104,8 @@ __device__ __forceinline__ unsigned long long global_timer() {
 
 // Bounded wait for the phase of `bar` with the given parity to complete.  Returns false
 // when the CTA is aborting or the limit ran out (then the error word and abort flag are set).
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                        int* err, int where) {
-  if (mbar_try(bar, parity)) return true;
   const unsigned long long t0 = global_timer();
   while (true) {
     if (mbar_try(bar, parity)) return true;
@@ -116,6 +116,27 @@ __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile i
       return false;
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          int* err, int where) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  if (ok) return true;
+  return mbar_wait_slow(bar, parity, abort_flag, err, where);
+}
+
+// Whole-warp wait: every lane waits, and the vote makes the outcome warp-uniform, so the
+// warp-collective issue helpers after it always run with the full warp.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity,
+                                               volatile int* abort_flag, int* err, int where) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, err, where));
 }
 
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* tm, int x, int y,
@@ -283,26 +304,26 @@ __device__ __forceinline__ TileRef tile_ref(const AttnParams& p, int t) {
 
 struct Bars {
   uint64_t q_full[2];
-  uint64_t s_full[2][2];   // [query tile g][buffer b]: S_j (j % 2 == b) landed in TMEM
-  uint64_t s_free[2][2];   // the softmax warps have read S_j
-  uint64_t p_full[2][2];   // P_j written to TMEM (and O rescaled if needed)
-  uint64_t pv_done[2][2];  // PV_j finished: P buffer b and O are free again
+  uint64_t s_full[2];    // per query tile g: S_j landed in TMEM
+  uint64_t s_free[2];    // per g: the softmax warps have read S_j
+  uint64_t p_full[2];    // per g: P_j written to TMEM (and O rescaled if needed)
+  uint64_t pv_done[2];   // per g: PV_j finished (P buffer and O are free again)
   uint64_t drain[2];
-  uint64_t kv_full[8];
-  uint64_t kv_empty[8];    // one arrival per active query tile
+  uint64_t kv_full[4];
+  uint64_t kv_empty[4];  // one arrival per active query tile
   uint32_t tmem_base;
   int abort_flag;
 };
 
-// Tensor-memory columns of query tile g (256 columns at 256 g), double-buffered:
-// head_dim 64:  S_b [64b, 64b+64), P_b [128+32b, 160+32b), O [192, 256);
-// head_dim 128: S_b [64b, 64b+64), P_b written over S_b [64b, 64b+32), O [128, 256).
+// Per-tile softmax state of one query row, and the TMEM column map of query tile g.
 template <int D>
 struct TmemMap {
+  // 256 columns per query tile: S [0,128); D = 64: P [128,192), O [192,256);
+  // D = 128: O [128,256) and P overwrites S [0,64) once S has been read into registers.
+  static constexpr uint32_t S = 0;
+  static constexpr uint32_t P = D == 64 ? 128 : 0;
+  static constexpr uint32_t O = D == 64 ? 192 : 128;
   static constexpr bool kPAliasesS = D != 64;
-  __host__ __device__ static constexpr uint32_t S(int b) { return 64u * b; }
-  __host__ __device__ static constexpr uint32_t P(int b) { return kPAliasesS ? 64u * b : 128u + 32u * b; }
-  static constexpr uint32_t O = D == 64 ? 192u : 128u;
 };
 
 template <int D>
@@ -316,7 +337,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   Bars* bars = reinterpret_cast<Bars*>(smem + C::OFF_BAR);
   volatile int* abort_flag = &bars->abort_flag;
 
-  const int warp = threadIdx.x >> 5;
+  // warp index through a shuffle: provably warp-uniform, so role-dependent descriptors and
+  // addresses stay in uniform registers (no per-instruction conversion before tcgen05.mma)
+  const int warp = __shfl_sync(0xffffffffu, (int)(threadIdx.x >> 5), 0);
   const int lane = threadIdx.x & 31;
   const int q_tiles = (p.tokens + BM - 1) / BM;
   const int tile0 = 2 * blockIdx.x;                 // this CTA's query tiles: tile0, tile0+1
@@ -335,13 +358,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int g = 0; g < 2; ++g) {
       mbar_init(bar(bars->q_full[g]), 1);
+      mbar_init(bar(bars->s_full[g]), 1);
+      mbar_init(bar(bars->s_free[g]), 128);
+      mbar_init(bar(bars->p_full[g]), 128);
+      mbar_init(bar(bars->pv_done[g]), 1);
       mbar_init(bar(bars->drain[g]), 1);
-      for (int b = 0; b < 2; ++b) {
-        mbar_init(bar(bars->s_full[g][b]), 1);
-        mbar_init(bar(bars->s_free[g][b]), 128);
-        mbar_init(bar(bars->p_full[g][b]), 128);
-        mbar_init(bar(bars->pv_done[g][b]), 1);
-      }
     }
     for (int s = 0; s < C::NS; ++s) {
       mbar_init(bar(bars->kv_full[s]), 1);
@@ -360,34 +381,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = bars->tmem_base;
-
+  const uint32_t tmem = __shfl_sync(0xffffffffu, bars->tmem_base, 0);
+  if (warp < 4) {
   if (warp == 0) {
     // ---------------- TMA producer (whole warp, elected lane issues) ----------------
     {
       int issued = 0;
       for (int g = 0; g < n_q; ++g) {
-        mbar_expect_tx(bar(bars->q_full[g]), C::Q_BYTES);
+        mbar_expect_tx(bar(bars->q_full[g]), C::TILE_BYTES);
 #pragma unroll
         for (int a = 0; a < C::ATOMS; ++a)
-          tma_load_3d(sQ + g * C::Q_BYTES + a * C::Q_ATOM, &p.tm_q, 64 * a, head,
+          tma_load_3d(sQ + g * C::TILE_BYTES + a * C::ATOM_BYTES, &p.tm_q, 64 * a, head,
                       (tile0 + g) * BM, bar(bars->q_full[g]));
       }
       for (int j = 0; j < n; ++j) {
         const int s = j % C::NS;
-        if (j >= C::NS && !__all_sync(kFull, mbar_wait(bar(bars->kv_empty[s]),
-                                                       ((j - C::NS) / C::NS) & 1, abort_flag,
-                                                       p.err, 1)))
+        if (j >= C::NS &&
+            !mbar_wait_warp(bar(bars->kv_empty[s]), ((j - C::NS) / C::NS) & 1, abort_flag, p.err, 1))
           break;
         const TileRef t = tile_ref(p, t_begin + j);
         const CUtensorMap* tk = t.special ? &p.tm_ks : &p.tm_kp;
         const CUtensorMap* tv = t.special ? &p.tm_vs : &p.tm_vp;
-        mbar_expect_tx(bar(bars->kv_full[s]), 2 * C::KV_BYTES);
+        mbar_expect_tx(bar(bars->kv_full[s]), 2 * C::TILE_BYTES);
 #pragma unroll
         for (int a = 0; a < C::ATOMS; ++a) {
-          tma_load_3d(sK + s * C::KV_BYTES + a * C::KV_ATOM, tk, 64 * a, t.row0, head,
+          tma_load_3d(sK + s * C::TILE_BYTES + a * C::ATOM_BYTES, tk, 64 * a, t.row0, head,
                       bar(bars->kv_full[s]));
-          tma_load_3d(sV + s * C::KV_BYTES + a * C::KV_ATOM, tv, 64 * a, t.row0, head,
+          tma_load_3d(sV + s * C::TILE_BYTES + a * C::ATOM_BYTES, tv, 64 * a, t.row0, head,
                       bar(bars->kv_full[s]));
         }
         ++issued;
@@ -413,96 +433,91 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (g < n_q) {  // whole warp, elected lane issues
       constexpr uint32_t idesc_s = idesc_bf16(BM, BN, false);
       constexpr uint32_t idesc_o = idesc_bf16(BM, D, true);
-      const uint32_t tG = tmem + 256 * g;
-      const uint32_t q_base = sQ + g * C::Q_BYTES;
-      bool ok = __all_sync(kFull, mbar_wait(bar(bars->q_full[g]), 0, abort_flag, p.err, 2));
+      const uint32_t tS = tmem + 256 * g + TM::S;
+      const uint32_t tP = tmem + 256 * g + TM::P;
+      const uint32_t tO = tmem + 256 * g + TM::O;
+      const uint32_t q_base = sQ + g * C::TILE_BYTES;
+      bool ok = mbar_wait_warp(bar(bars->q_full[g]), 0, abort_flag, p.err, 2);
       tc_fence_after();
       auto issue_qk = [&](int j) -> bool {
         const int s = j % C::NS;
-        const int b = j & 1;
-        if (!__all_sync(kFull, mbar_wait(bar(bars->kv_full[s]), (j / C::NS) & 1, abort_flag, p.err, 4)))
+        if (!mbar_wait_warp(bar(bars->kv_full[s]), (j / C::NS) & 1, abort_flag, p.err, 4))
           return false;
-        // S buffer b held S_{j-2} (and, with head_dim 128, P_{j-2}): wait until it is free
-        if (j >= 2 && !__all_sync(kFull, mbar_wait(TM::kPAliasesS ? bar(bars->pv_done[g][b])
-                                                                  : bar(bars->s_free[g][b]),
-                                                   ((j - 2) >> 1) & 1, abort_flag, p.err, 5)))
+        if (j >= 1 && !mbar_wait_warp(bar(bars->s_free[g]), (j - 1) & 1, abort_flag, p.err, 5))
           return false;
         tc_fence_after();
-        const uint32_t k_base = sK + s * C::KV_BYTES;
+        const uint32_t k_base = sK + s * C::TILE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t in_atom = (kk & 3) * 32;
-          mma_ss(tG + TM::S(b), sdesc(q_base + (kk >> 2) * C::Q_ATOM + in_atom, 16, 1024),
-                 sdesc(k_base + (kk >> 2) * C::KV_ATOM + in_atom, 16, 1024), idesc_s,
+          const uint32_t off = (kk >> 2) * C::ATOM_BYTES + (kk & 3) * 32;
+          mma_ss(tS, sdesc(q_base + off, 16, 1024), sdesc(k_base + off, 16, 1024), idesc_s,
                  kk > 0 ? 1u : 0u);
         }
-        mma_commit(bar(bars->s_full[g][b]));
+        mma_commit(bar(bars->s_full[g]));
         return true;
       };
       auto issue_pv = [&](int i) -> bool {
-        const int b = i & 1;
-        if (!__all_sync(kFull, mbar_wait(bar(bars->p_full[g][b]), (i >> 1) & 1, abort_flag,
-                                         p.err, 3)))
-          return false;
+        if (!mbar_wait_warp(bar(bars->p_full[g]), i & 1, abort_flag, p.err, 3)) return false;
         tc_fence_after();
         const int s = i % C::NS;
-        const uint32_t v_base = sV + s * C::KV_BYTES;
+        const uint32_t v_base = sV + s * C::TILE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
           // B = V tile [keys][D], MN-major: 16 keys = 2 groups of 8 rows of 128 B
-          const uint64_t bd = sdesc(v_base + kk * 2048, C::KV_ATOM, 1024);
-          mma_ts(tG + TM::O, tG + TM::P(b) + 8 * kk, bd, idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
+          const uint64_t bd = sdesc(v_base + kk * 2048, C::ATOM_BYTES, 1024);
+          mma_ts(tO, tP + 8 * kk, bd, idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit(bar(bars->pv_done[g][b]));
+        mma_commit(bar(bars->pv_done[g]));
         mma_commit(bar(bars->kv_empty[s]));
         return true;
       };
       if (ok && n > 0) ok = issue_qk(0);
-      if (ok && n > 1) ok = issue_qk(1);
-      for (int i = 0; ok && i < n; ++i) {
+      for (int j = 1; ok && j < n; ++j) {
         if (TM::kPAliasesS) {
-          // S_{i+2} overwrites P_i: issue PV_i first (issue_qk waits for it to finish)
-          ok = issue_pv(i) && (i + 2 >= n || issue_qk(i + 2));
+          // P_{j-1} lives in S: PV_{j-1} must have read it before S_j overwrites it
+          ok = issue_pv(j - 1) &&
+               mbar_wait_warp(bar(bars->pv_done[g]), (j - 1) & 1, abort_flag, p.err, 10) &&
+               issue_qk(j);
         } else {
-          // S_{i+2} only needs S_i read: issue it first so the softmax never waits for S
-          ok = (i + 2 >= n || issue_qk(i + 2)) && issue_pv(i);
+          // S_j only needs S_{j-1} read: issue it first so the softmax can start early
+          ok = issue_qk(j) && issue_pv(j - 1);
         }
       }
+      if (ok && !*abort_flag && n > 0) issue_pv(n - 1);
       // every MMA issued by this thread has completed once `drain` flips
       mma_commit(bar(bars->drain[g]));
       const unsigned long long t0 = global_timer();
       while (!mbar_try(bar(bars->drain[g]), 0) && global_timer() - t0 < kWaitLimitNs) {
       }
     }
-  } else if (warp >= 4) {
+  }
+  } else {
     // ---------------- softmax + epilogue: warps 4..7 tile 0, warps 8..11 tile 1 ----------------
     const int g = (warp - 4) >> 2;
     const int quad = warp & 3;                  // TMEM lane quadrant this warp may access
     const int row = (tile0 + g) * BM + quad * 32 + lane;
     const uint32_t lane_base = tmem + 256 * g + ((uint32_t)(quad * 32) << 16);
+    const uint32_t tS = lane_base + TM::S;
+    const uint32_t tP = lane_base + TM::P;
     const uint32_t tO = lane_base + TM::O;
     float m = -INFINITY;  // running max (log2 domain) the P values and O are relative to
     float l = 0.f;
     bool ok = g < n_q;
     uint32_t S[BN];
     for (int j = 0; ok && j < n; ++j) {
-      const int b = j & 1;
       // every wait in these warps is made warp-uniform, so warp-collective tcgen05 ops and
       // votes below always run with the whole warp
-      if (!__all_sync(kFull, mbar_wait(bar(bars->s_full[g][b]), (j >> 1) & 1, abort_flag,
-                                       p.err, 6))) {
+      if (!__all_sync(kFull, mbar_wait(bar(bars->s_full[g]), j & 1, abort_flag, p.err, 6))) {
         ok = false;
         break;
       }
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < BN / 32; ++c) tmem_ld32(lane_base + TM::S(b) + 32 * c, S + 32 * c);
+      for (int c = 0; c < BN / 32; ++c) tmem_ld32(tS + 32 * c, S + 32 * c);
       tmem_wait_ld();
       reg_fence<BN>(S);
-      if (!TM::kPAliasesS) {
-        tc_fence_before();
-        mbar_arrive(bar(bars->s_free[g][b]));
-      }
+      tc_fence_before();
+      mbar_arrive(bar(bars->s_free[g]));
 
       const int valid = tile_ref(p, t_begin + j).valid;
       if (valid != BN) {
@@ -530,33 +545,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         l *= alpha;
         rescale = true;
       }
-      // P_j reuses P buffer b, last read by PV_{j-2} (head_dim 64; with head_dim 128 the
-      // buffer is S_b, and S_j could only be computed after PV_{j-2} finished)
-      if (!TM::kPAliasesS && j >= 2 &&
-          !__all_sync(kFull, mbar_wait(bar(bars->pv_done[g][b]), ((j - 2) >> 1) & 1,
-                                       abort_flag, p.err, 7))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
+      // exponentials first, into registers (packed over S), so that the wait for PV_{j-1}
+      // below overlaps this work instead of stalling in front of it
       const uint64_t c2 = pack_f2(p.scale_log2, p.scale_log2);
       const uint64_t nm2 = pack_f2(-m, -m);
       uint64_t l4[4] = {0, 0, 0, 0};
 #pragma unroll
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int i0 = 32 * c + 2 * i;
-          float x0, x1;
-          unpack_f2(ffma2(pack_f2(__uint_as_float(S[i0]), __uint_as_float(S[i0 + 1])), c2, nm2),
-                    x0, x1);
-          const float p0 = fast_exp2(x0);
-          const float p1 = fast_exp2(x1);
-          l4[i & 3] = fadd2(l4[i & 3], pack_f2(p0, p1));
-          pk[i] = pack_bf16(p0, p1);
-        }
-        tmem_st16(lane_base + TM::P(b) + 16 * c, pk);
+      for (int i = 0; i < BN / 2; ++i) {
+        float x0, x1;
+        unpack_f2(ffma2(pack_f2(__uint_as_float(S[2 * i]), __uint_as_float(S[2 * i + 1])), c2,
+                        nm2),
+                  x0, x1);
+        const float p0 = fast_exp2(x0);
+        const float p1 = fast_exp2(x1);
+        l4[i & 3] = fadd2(l4[i & 3], pack_f2(p0, p1));
+        S[i] = pack_bf16(p0, p1);  // S[0 .. BN/2) now holds P_j as bf16 pairs
       }
       {
         float a0, a1, b0, b1, c0, c1, d0, d1;
@@ -566,14 +569,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         unpack_f2(l4[3], d0, d1);
         l += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
       }
+      // P_j overwrites P_{j-1} (and O may be rescaled): PV_{j-1} must have finished
+      if (j >= 1 && !__all_sync(kFull, mbar_wait(bar(bars->pv_done[g]), (j - 1) & 1,
+                                                 abort_flag, p.err, 7))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < BN / 32; ++c) tmem_st16(tP + 16 * c, S + 16 * c);
       if (__any_sync(kFull, rescale) && j > 0) {
         // O holds sum_{i<j} P_i V_i relative to the old max: scale it before PV_j lands
-        if (!__all_sync(kFull, mbar_wait(bar(bars->pv_done[g][(j - 1) & 1]), ((j - 1) >> 1) & 1,
-                                         abort_flag, p.err, 8))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
@@ -588,11 +594,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(bars->p_full[g][b]));
+      mbar_arrive(bar(bars->p_full[g]));
     }
     if (ok && n > 0 &&
-        __all_sync(kFull, mbar_wait(bar(bars->pv_done[g][(n - 1) & 1]), ((n - 1) >> 1) & 1,
-                                    abort_flag, p.err, 9))) {
+        __all_sync(kFull, mbar_wait(bar(bars->pv_done[g]), (n - 1) & 1, abort_flag, p.err, 9))) {
       tc_fence_after();
       const float inv_l = 1.f / l;
       const bool store = row < p.tokens;

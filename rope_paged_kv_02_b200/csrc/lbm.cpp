@@ -50,7 +50,7 @@ struct lbm_cache {
 namespace {
 
 constexpr int kMaxSplits = 16;
-constexpr int kKeyTile = 64;  // keys per attention key tile (page strides are multiples)
+constexpr int kKeyTile = 128;  // keys per attention key tile (page strides are multiples)
 
 int elem_size(int dtype) { return dtype == LBM_BF16 ? 2 : 4; }
 
@@ -115,7 +115,7 @@ int plan_splits(int work_units, int n_tiles, int num_sms, double combine_tiles_p
     if (s_eff != s) continue;
     const long long units = (long long)work_units * s;
     const long long waves = (units + num_sms - 1) / num_sms;
-    double cost = (double)waves * (tps + 8.0);
+    double cost = (double)waves * (tps + 4.0);
     if (s > 1) cost += 8.0 + combine_tiles_per_split * s;
     if (cost < best_cost - 1e-9) {
       best_cost = cost;
@@ -376,8 +376,8 @@ int lbm_attend_frame(lbm_cache_t* c, const void* q, void* out, void* stream) {
     p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)c->head_dim));
     for (size_t i = 0; i < pages.size(); ++i) p.pages[i] = (uint16_t)pages[i];
     const int q_tiles = (T + 127) / 128;
-    // combine cost of one split, in key-tile times (a tile of both query tiles ~0.5 us)
-    const double combine = (double)T * c->heads * c->head_dim * 4.0 / 3.0e6;
+    // combine cost of one split, in key-tile times (a tile of both query tiles ~1 us)
+    const double combine = (double)T * c->heads * c->head_dim * 4.0 / 6.0e6;
     p.n_splits = plan_splits((q_tiles + 1) / 2 * c->heads, p.n_tiles, c->num_sms, combine,
                              c->max_splits);
     if (c->forced_splits) p.n_splits = std::min(c->forced_splits, p.n_tiles);

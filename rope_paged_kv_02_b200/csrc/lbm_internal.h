@@ -26,7 +26,7 @@ struct Pools {
   void* k_special;
   void* v_special;
   int num_pages;
-  int page_stride;  // tokens per page slot (patches_per_frame rounded up to 64)
+  int page_stride;  // tokens per page slot (patches_per_frame rounded up to 128)
   int spec_cap;     // special stream capacity in tokens (multiple of 128)
 };
 
@@ -58,10 +58,10 @@ struct AttnParams {
   int heads;
   int patches;           // valid tokens per patch page
   int page_stride;
-  int tiles_per_page;    // key tiles per patch page: ceil(patches / 64)
+  int tiles_per_page;    // key tiles per patch page: ceil(patches / 128)
   int n_pages;           // visible patch pages
   int n_special;         // visible special tokens
-  int n_tiles;           // n_pages * tiles_per_page + ceil(n_special / 64)
+  int n_tiles;           // n_pages * tiles_per_page + ceil(n_special / 128)
   int tiles_per_split;
   int n_splits;
   float scale_log2;      // log2(e) / sqrt(head_dim)
