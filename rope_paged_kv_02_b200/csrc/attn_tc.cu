@@ -545,21 +545,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         l *= alpha;
         rescale = true;
       }
-      // exponentials first, into registers (packed over S), so that the wait for PV_{j-1}
-      // below overlaps this work instead of stalling in front of it
+      // P_j overwrites P_{j-1} (and O may be rescaled): PV_{j-1} must have finished
+      if (j >= 1 && !__all_sync(kFull, mbar_wait(bar(bars->pv_done[g]), (j - 1) & 1,
+                                                 abort_flag, p.err, 7))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
       const uint64_t c2 = pack_f2(p.scale_log2, p.scale_log2);
       const uint64_t nm2 = pack_f2(-m, -m);
       uint64_t l4[4] = {0, 0, 0, 0};
 #pragma unroll
-      for (int i = 0; i < BN / 2; ++i) {
-        float x0, x1;
-        unpack_f2(ffma2(pack_f2(__uint_as_float(S[2 * i]), __uint_as_float(S[2 * i + 1])), c2,
-                        nm2),
-                  x0, x1);
-        const float p0 = fast_exp2(x0);
-        const float p1 = fast_exp2(x1);
-        l4[i & 3] = fadd2(l4[i & 3], pack_f2(p0, p1));
-        S[i] = pack_bf16(p0, p1);  // S[0 .. BN/2) now holds P_j as bf16 pairs
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int i0 = 32 * c + 2 * i;
+          float x0, x1;
+          unpack_f2(ffma2(pack_f2(__uint_as_float(S[i0]), __uint_as_float(S[i0 + 1])), c2, nm2),
+                    x0, x1);
+          const float p0 = fast_exp2(x0);
+          const float p1 = fast_exp2(x1);
+          l4[i & 3] = fadd2(l4[i & 3], pack_f2(p0, p1));
+          pk[i] = pack_bf16(p0, p1);
+        }
+        tmem_st16(tP + 16 * c, pk);
       }
       {
         float a0, a1, b0, b1, c0, c1, d0, d1;
@@ -569,15 +579,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         unpack_f2(l4[3], d0, d1);
         l += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
       }
-      // P_j overwrites P_{j-1} (and O may be rescaled): PV_{j-1} must have finished
-      if (j >= 1 && !__all_sync(kFull, mbar_wait(bar(bars->pv_done[g]), (j - 1) & 1,
-                                                 abort_flag, p.err, 7))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < BN / 32; ++c) tmem_st16(tP + 16 * c, S + 16 * c);
       if (__any_sync(kFull, rescale) && j > 0) {
         // O holds sum_{i<j} P_i V_i relative to the old max: scale it before PV_j lands
 #pragma unroll
