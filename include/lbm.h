@@ -142,6 +142,26 @@ LBM_API int lbm_append_frame(lbm_cache_t* cache, void* q, const void* k, const v
  * CTAs.  Errors: LBM_ERR_SEQUENCE if no frame is pending. */
 LBM_API int lbm_attend_frame(lbm_cache_t* cache, const void* q, void* out, void* stream);
 
+/* Like lbm_attend_frame, for callers that may not allocate device memory while frames
+ * stream (a runtime that owns the whole GPU through its own pool and budget, or a real-time
+ * loop where cudaMalloc / cudaFree would synchronise the device).  The pages describe no such
+ * call; it has no counterpart there.  Same arguments, same result and same page-table update
+ * as lbm_attend_frame, but the split-KV partial results go to a file-scope device array of
+ * LBM_NOALLOC_SCRATCH_BYTES (16 MiB) that every GPU loading the library holds until exit,
+ * instead of the cache's own scratch; the call allocates nothing (device or host heap).
+ *   - bf16 caches only (LBM_ERR_UNSUPPORTED otherwise).
+ *   - The first call on a device looks up the array's device address with that device
+ *     current; make that first call before any stream capture.
+ *   - A frame whose planned key split needs more than LBM_NOALLOC_SCRATCH_BYTES of partial
+ *     results (splits x T x heads x (head_dim + 1) x 4 bytes) is refused with
+ *     LBM_ERR_CAPACITY and the cache is left as it was.
+ *   - Every call shares the array and leaves its last contents there; nothing in it needs
+ *     to start at zero.  Calls whose kernels overlap on the GPU (several streams or caches
+ *     at once) race on it: order them. */
+#define LBM_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+LBM_API int lbm_attend_frame_noalloc(lbm_cache_t* cache, const void* q, void* out,
+                                     void* stream);
+
 /* Forget every frame: all pages free, special stream empty ([KVBenefits] "Cross-Window
  * Alignment for Long Videos": clean_kv_cache).  Host-only; pool contents are left as they
  * are (nothing reads them before they are written again). */

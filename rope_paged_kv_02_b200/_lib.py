@@ -33,7 +33,8 @@ LBM_MAX_PAGES = 1024
 # every symbol include/lbm.h declares
 SYMBOLS = [
     "lbm_rope3d_tables", "lbm_rope3d_expand", "lbm_rope_destroy",
-    "lbm_cache_create", "lbm_append_frame", "lbm_attend_frame", "lbm_cache_reset",
+    "lbm_cache_create", "lbm_append_frame", "lbm_attend_frame", "lbm_attend_frame_noalloc",
+    "lbm_cache_reset",
     "lbm_cache_state", "lbm_cache_read_kv", "lbm_cache_check", "lbm_cache_destroy",
     "lbm_status_string",
     "lbm_pager_create", "lbm_pager_append", "lbm_pager_visible", "lbm_pager_finish",
@@ -85,6 +86,7 @@ def load() -> ctypes.CDLL:
     lib.lbm_cache_create.argtypes = [c_int] * 8 + [c_void, ctypes.POINTER(c_void)]
     lib.lbm_append_frame.argtypes = [c_void, c_void, c_void, c_void, c_ll, c_int, c_void]
     lib.lbm_attend_frame.argtypes = [c_void, c_void, c_void, c_void]
+    lib.lbm_attend_frame_noalloc.argtypes = [c_void, c_void, c_void, c_void]
     lib.lbm_cache_reset.argtypes = [c_void]
     lib.lbm_cache_state.argtypes = [c_void, ctypes.POINTER(CacheState)]
     lib.lbm_cache_read_kv.argtypes = [c_void, c_int, c_int, c_int, c_void]

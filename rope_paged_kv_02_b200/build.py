@@ -17,7 +17,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "liblbm.so")
-SOURCES = ["pager.cpp", "rope.cu", "attn_tc.cu", "attn_simt.cu", "lbm.cpp"]
+SOURCES = ["pager.cpp", "rope.cu", "attn_tc.cu", "attn_simt.cu", "attn_static.cu", "lbm.cpp"]
 HEADERS = ["pager.h", "lbm_internal.h"]
 
 NVCC = os.environ.get("NVCC", "nvcc")

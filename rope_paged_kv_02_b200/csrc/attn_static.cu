@@ -1,0 +1,47 @@
+// Split-KV scratch that lives in a file-scope device array, for lbm_attend_frame_noalloc.
+//
+// Some callers of this library may not allocate device memory while frames stream: a
+// serving runtime that owns every byte of the GPU through its own pool and budget, or a
+// real-time frame loop where cudaMalloc / cudaFree would synchronise the device and stall
+// the stream.  lbm_attend_frame_noalloc serves them: its split-KV partial results go to the
+// array below, which the CUDA runtime places when the library is loaded, so the call itself
+// allocates nothing.
+//
+// The array is shared by every call on a device and keeps the last call's contents.  No
+// part of it needs to start at zero: each call writes every partial row it later reads.
+// Calls that overlap on the GPU (two streams, or two caches at once) race on it.
+#include "../../include/lbm.h"
+#include "lbm_internal.h"
+
+namespace lbm {
+namespace {
+
+constexpr size_t kNoallocScratchFloats = LBM_NOALLOC_SCRATCH_BYTES / sizeof(float);
+
+static __device__ __align__(256) float g_noalloc_scratch[kNoallocScratchFloats];
+
+constexpr int kMaxDevices = 64;
+float* g_scratch_ptr[kMaxDevices];  // device address of the array, per device, once set
+bool g_scratch_ready[kMaxDevices];
+
+}  // namespace
+
+// Device address of the scratch array on `device`, which must be the current device.  The
+// first call on a device looks the address up (cudaGetSymbolAddress) and remembers it.
+int noalloc_scratch(int device, float** ptr, size_t* floats) {
+  if (device < 0 || device >= kMaxDevices || !ptr || !floats) return LBM_ERR_INVALID;
+  if (!g_scratch_ready[device]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return LBM_ERR_CUDA;
+    }
+    g_scratch_ptr[device] = static_cast<float*>(p);
+    g_scratch_ready[device] = true;
+  }
+  *ptr = g_scratch_ptr[device];
+  *floats = kNoallocScratchFloats;
+  return LBM_OK;
+}
+
+}  // namespace lbm

@@ -419,6 +419,72 @@ int lbm_attend_frame(lbm_cache_t* c, const void* q, void* out, void* stream) {
   return LBM_OK;
 }
 
+int lbm_attend_frame_noalloc(lbm_cache_t* c, const void* q, void* out, void* stream) {
+  if (!c || !q || !out || !aligned16(q) || !aligned16(out)) return LBM_ERR_INVALID;
+  if (c->dtype != LBM_BF16) return LBM_ERR_UNSUPPORTED;
+  if (!c->pager.pending()) return LBM_ERR_SEQUENCE;
+  if (use_device(c->device) != LBM_OK) return LBM_ERR_CUDA;
+  float* scratch = nullptr;
+  size_t scratch_floats = 0;
+  const int st = lbm::noalloc_scratch(c->device, &scratch, &scratch_floats);
+  if (st != LBM_OK) return st;
+  lbm::AttnParams p;  // on the stack: this call touches no heap
+  // visible pages in page-table order, built without a container
+  int n_pages = 0;
+  for (const auto& e : c->pager.scale()) p.pages[n_pages++] = (uint16_t)e.page;
+  for (const auto& e : c->pager.window()) p.pages[n_pages++] = (uint16_t)e.page;
+  p.pages[n_pages++] = (uint16_t)c->pager.pending_page();
+  const int n_sp = c->pager.n_special() + c->psi;
+  const int T = c->psi + c->patches;
+  const uint64_t row = (uint64_t)c->head_dim * 2;
+  if (q != c->tm_q_ptr) {
+    if (!make_map(&c->tm_q, q, c->head_dim, c->heads, T, row, row * c->heads, 1, 128))
+      return LBM_ERR_CUDA;
+    c->tm_q_ptr = q;
+  }
+  p.tm_q = c->tm_q;
+  p.tm_kp = c->tm_kp;
+  p.tm_vp = c->tm_vp;
+  p.tm_ks = c->tm_ks;
+  p.tm_vs = c->tm_vs;
+  p.out = out;
+  p.err = c->d_err;
+  p.tokens = T;
+  p.heads = c->heads;
+  p.patches = c->patches;
+  p.page_stride = c->pools.page_stride;
+  p.tiles_per_page = (c->patches + kKeyTile - 1) / kKeyTile;
+  p.n_pages = n_pages;
+  p.n_special = n_sp;
+  p.n_tiles = p.n_pages * p.tiles_per_page + (n_sp + kKeyTile - 1) / kKeyTile;
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)c->head_dim));
+  const int q_tiles = (T + 127) / 128;
+  const double combine = (double)T * c->heads * c->head_dim * 4.0 / 6.0e6;
+  p.n_splits = plan_splits((q_tiles + 1) / 2 * c->heads, p.n_tiles, c->num_sms, combine,
+                           c->max_splits);
+  if (c->forced_splits) p.n_splits = std::min(c->forced_splits, p.n_tiles);
+  p.tiles_per_split = (p.n_tiles + p.n_splits - 1) / p.n_splits;
+  p.n_splits = (p.n_tiles + p.tiles_per_split - 1) / p.tiles_per_split;
+  const size_t rows = (size_t)p.n_splits * T * c->heads;
+  if (p.n_splits > 1 && rows * (c->head_dim + 1) > scratch_floats) return LBM_ERR_CAPACITY;
+  p.part_o = scratch;
+  p.part_lse = scratch + rows * c->head_dim;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  order_before(c, s);
+  if (lbm::launch_attn_tc(p, c->head_dim, q_tiles, s) != cudaSuccess) return LBM_ERR_CUDA;
+  ++c->launches;
+  if (p.n_splits > 1) {
+    if (lbm::launch_attn_combine(p.part_o, p.part_lse, out, p.n_splits, T, c->heads,
+                                 c->head_dim, s) != cudaSuccess)
+      return LBM_ERR_CUDA;
+    ++c->launches;
+  }
+  order_after(c, s);
+  int evicted = -1;
+  c->pager.finish(&evicted);
+  return LBM_OK;
+}
+
 int lbm_cache_reset(lbm_cache_t* c) {
   if (!c) return LBM_ERR_INVALID;
   c->pager.reset();

@@ -95,6 +95,9 @@ cudaError_t launch_attn_combine(const float* part_o, const float* part_lse, void
                                 int n_splits, int tokens, int heads, int head_dim,
                                 cudaStream_t s);
 
+// attn_static.cu: device address of the file-scope split-KV scratch on `device` (current)
+int noalloc_scratch(int device, float** ptr, size_t* floats);
+
 // attn_simt.cu (fp32)
 cudaError_t launch_attn_simt(const SimtParams& p, cudaStream_t s);
 
