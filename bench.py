@@ -49,6 +49,30 @@ def _peaks():
             "source": "fallback"}
 
 
+def measured_traffic(avg_keys: float):
+    """DRAM bytes per attention launch from the committed ncu summary, scaled from the
+    captured frame's key count to the stream's average (K/V reads dominate and grow with
+    the keys); None once the kernel source differs from the one that was profiled."""
+    import hashlib
+    prof = os.path.join(ROOT, "profiles", "attn_tc_stream768.md")
+    src = os.path.join(ROOT, "rope_paged_kv_02_b200", "csrc", "attn_tc.cu")
+    if not os.path.exists(prof):
+        return None
+    fields = {}
+    for line in open(prof):
+        if ":" in line and not line.startswith("|"):
+            k, v = line.split(":", 1)
+            fields[k.strip()] = v.strip()
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    if fields.get("kernel_source_sha256_16") != sha:
+        return None
+    try:
+        return float(fields["traffic_bytes_per_launch"]) * avg_keys / float(
+            fields["algorithmic_keys_of_capture"])
+    except (KeyError, ValueError):
+        return None
+
+
 def frame_work(cfg):
     """Algorithmic work per frame of a stream: (attention FLOPs, append bytes, keys seen).
 
@@ -342,7 +366,7 @@ def main():
     append_ms = np.array([[e[0].elapsed_time(e[1]) for e in st] for st in evs])
     attn_ms = np.array([[e[1].elapsed_time(e[2]) for e in st] for st in evs])
 
-    flops, nbytes, _ = frame_work(cfg)
+    flops, nbytes, keys = frame_work(cfg)
     frames_total = F * args.steps * world
     value = frames_total / (ms_max / 1e3)
     peaks = _peaks()
@@ -365,7 +389,8 @@ def main():
         "roofline": {
             "bound": "tensor", "achieved": attn_tflops,
             "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-            "frac": attn_tflops / peaks["bf16_tflops_sustained"], "traffic": None,
+            "frac": attn_tflops / peaks["bf16_tflops_sustained"],
+            "traffic": measured_traffic(float(keys.mean())) if args.config == 1 else None,
             "kernel": "paged attention (attn_tc + split-KV combine), all frames",
             "peak_source": peaks["source"] + " bf16_tflops_sustained",
             "steady_state_achieved": ss_tflops,
