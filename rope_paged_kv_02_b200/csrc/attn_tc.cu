@@ -303,29 +303,54 @@ __device__ __forceinline__ TileRef tile_ref(const AttnParams& p, int t) {
 }
 
 struct Bars {
-  uint64_t q_full[2];
-  uint64_t s_full[2];    // per query tile g: S_j landed in TMEM
-  uint64_t s_free[2];    // per g: the softmax warps have read S_j
-  uint64_t p_full[2];    // per g: P_j written to TMEM (and O rescaled if needed)
-  uint64_t pv_done[2];   // per g: PV_j finished (P buffer and O are free again)
+  uint64_t q_full;         // the query tiles of the current segment landed
+  uint64_t q_empty;        // both MMA issuers are done with them (count 2)
+  uint64_t s_full[2];      // per query tile g: S_j landed in TMEM
+  uint64_t s_free[2];      // per g: the softmax warps have read S_j
+  uint64_t p_full[2];      // per g: P_j written to TMEM (and O rescaled if needed)
+  uint64_t pv_done[2];     // per g: PV_j finished (P buffer and O are free again)
+  uint64_t o_free[2];      // per g: the epilogue has read O of the segment
   uint64_t drain[2];
   uint64_t kv_full[4];
-  uint64_t kv_empty[4];  // one arrival per active query tile
+  uint64_t kv_empty[4];    // one arrival per MMA issuer (count 2)
   uint32_t tmem_base;
   int abort_flag;
 };
 
-// Per-tile softmax state of one query row, and the TMEM column map of query tile g.
+// Tensor-memory columns of query tile g (256 columns at 256 g): S [0,128); head_dim 64:
+// P [128,192), O [192,256); head_dim 128: O [128,256), P written over S [0,64) after S is
+// read into registers.
 template <int D>
 struct TmemMap {
-  // 256 columns per query tile: S [0,128); D = 64: P [128,192), O [192,256);
-  // D = 128: O [128,256) and P overwrites S [0,64) once S has been read into registers.
   static constexpr uint32_t S = 0;
   static constexpr uint32_t P = D == 64 ? 128 : 0;
   static constexpr uint32_t O = D == 64 ? 192 : 128;
   static constexpr bool kPAliasesS = D != 64;
 };
 
+// One run of key tiles of one unit, as a CTA walks its share of the work.
+struct Segment {
+  int unit, pair, head, a, b;   // key tiles [a, b) of unit (pair, head)
+  int n_q;                      // query tiles of the pair (1 for an odd last pair)
+  bool whole;                   // the segment is the whole unit: write the final output
+};
+
+__device__ __forceinline__ Segment segment_at(const AttnParams& p, long long x, long long hi,
+                                              int q_tiles) {
+  Segment sg;
+  sg.unit = (int)(x / p.n_tiles);
+  sg.pair = sg.unit % p.n_pairs;
+  sg.head = sg.unit / p.n_pairs;
+  sg.a = (int)(x - (long long)sg.unit * p.n_tiles);
+  const long long end = min(hi, (long long)(sg.unit + 1) * p.n_tiles);
+  sg.b = (int)(end - (long long)sg.unit * p.n_tiles);
+  sg.n_q = min(2, q_tiles - 2 * sg.pair);
+  sg.whole = sg.a == 0 && sg.b == p.n_tiles;
+  return sg;
+}
+
+// Persistent CTA c of p.grid walks the global work items [sk_lo(c), sk_lo(c+1)).  Every role
+// walks the same segments; barrier phases run on across segments (counters per role).
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ AttnParams p) {
@@ -338,17 +363,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = &bars->abort_flag;
 
   // warp index through a shuffle: provably warp-uniform, so role-dependent descriptors and
-  // addresses stay in uniform registers (no per-instruction conversion before tcgen05.mma)
+  // addresses stay in uniform registers
   const int warp = __shfl_sync(0xffffffffu, (int)(threadIdx.x >> 5), 0);
   const int lane = threadIdx.x & 31;
   const int q_tiles = (p.tokens + BM - 1) / BM;
-  const int tile0 = 2 * blockIdx.x;                 // this CTA's query tiles: tile0, tile0+1
-  const int n_q = min(2, q_tiles - tile0);          // 1 for an odd last pair
-  const int split = blockIdx.y;
-  const int head = blockIdx.z;
-  const int t_begin = split * p.tiles_per_split;
-  const int t_end = min(p.n_tiles, t_begin + p.tiles_per_split);
-  const int n = t_end - t_begin;
+  const long long lo = sk_lo(p.work, p.grid, blockIdx.x);
+  const long long hi = sk_lo(p.work, p.grid, blockIdx.x + 1);
 
   const uint32_t sQ = smem_u32(smem + C::OFF_Q);
   const uint32_t sK = smem_u32(smem + C::OFF_K);
@@ -356,17 +376,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar = [&](const uint64_t& b) { return smem_u32(&b); };
 
   if (threadIdx.x == 0) {
+    mbar_init(bar(bars->q_full), 1);
+    mbar_init(bar(bars->q_empty), 2);
     for (int g = 0; g < 2; ++g) {
-      mbar_init(bar(bars->q_full[g]), 1);
       mbar_init(bar(bars->s_full[g]), 1);
       mbar_init(bar(bars->s_free[g]), 128);
       mbar_init(bar(bars->p_full[g]), 128);
       mbar_init(bar(bars->pv_done[g]), 1);
+      mbar_init(bar(bars->o_free[g]), 128);
       mbar_init(bar(bars->drain[g]), 1);
     }
     for (int s = 0; s < C::NS; ++s) {
       mbar_init(bar(bars->kv_full[s]), 1);
-      mbar_init(bar(bars->kv_empty[s]), n_q);
+      mbar_init(bar(bars->kv_empty[s]), 2);
     }
     bars->abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -382,66 +404,106 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = __shfl_sync(0xffffffffu, bars->tmem_base, 0);
-  if (warp < 4) {
+
   if (warp == 0) {
     // ---------------- TMA producer (whole warp, elected lane issues) ----------------
-    {
-      int issued = 0;
-      for (int g = 0; g < n_q; ++g) {
-        mbar_expect_tx(bar(bars->q_full[g]), C::TILE_BYTES);
+    int issued = 0;        // key tiles issued so far (ring position)
+    int seg_i = 0;
+    bool ok = true;
+    for (long long x = lo; ok && x < hi; ++seg_i) {
+      const Segment sg = segment_at(p, x, hi, q_tiles);
+      x = (long long)sg.unit * p.n_tiles + sg.b;
+      // the query buffers are free once both MMA issuers are done with the last segment
+      if (seg_i > 0 &&
+          !mbar_wait_warp(bar(bars->q_empty), (seg_i - 1) & 1, abort_flag, p.err, 12)) {
+        ok = false;
+        break;
+      }
+      mbar_expect_tx(bar(bars->q_full), sg.n_q * C::TILE_BYTES);
+      for (int g = 0; g < sg.n_q; ++g) {
 #pragma unroll
         for (int a = 0; a < C::ATOMS; ++a)
-          tma_load_3d(sQ + g * C::TILE_BYTES + a * C::ATOM_BYTES, &p.tm_q, 64 * a, head,
-                      (tile0 + g) * BM, bar(bars->q_full[g]));
+          tma_load_3d(sQ + g * C::TILE_BYTES + a * C::ATOM_BYTES, &p.tm_q, 64 * a, sg.head,
+                      (2 * sg.pair + g) * BM, bar(bars->q_full));
       }
-      for (int j = 0; j < n; ++j) {
-        const int s = j % C::NS;
-        if (j >= C::NS &&
-            !mbar_wait_warp(bar(bars->kv_empty[s]), ((j - C::NS) / C::NS) & 1, abort_flag, p.err, 1))
+      for (int t = sg.a; t < sg.b; ++t, ++issued) {
+        const int s = issued % C::NS;
+        if (issued >= C::NS &&
+            !mbar_wait_warp(bar(bars->kv_empty[s]), ((issued - C::NS) / C::NS) & 1, abort_flag,
+                            p.err, 1)) {
+          ok = false;
           break;
-        const TileRef t = tile_ref(p, t_begin + j);
-        const CUtensorMap* tk = t.special ? &p.tm_ks : &p.tm_kp;
-        const CUtensorMap* tv = t.special ? &p.tm_vs : &p.tm_vp;
+        }
+        const TileRef tr = tile_ref(p, t);
+        const CUtensorMap* tk = tr.special ? &p.tm_ks : &p.tm_kp;
+        const CUtensorMap* tv = tr.special ? &p.tm_vs : &p.tm_vp;
         mbar_expect_tx(bar(bars->kv_full[s]), 2 * C::TILE_BYTES);
 #pragma unroll
         for (int a = 0; a < C::ATOMS; ++a) {
-          tma_load_3d(sK + s * C::TILE_BYTES + a * C::ATOM_BYTES, tk, 64 * a, t.row0, head,
+          tma_load_3d(sK + s * C::TILE_BYTES + a * C::ATOM_BYTES, tk, 64 * a, tr.row0, sg.head,
                       bar(bars->kv_full[s]));
-          tma_load_3d(sV + s * C::TILE_BYTES + a * C::ATOM_BYTES, tv, 64 * a, t.row0, head,
+          tma_load_3d(sV + s * C::TILE_BYTES + a * C::ATOM_BYTES, tv, 64 * a, tr.row0, sg.head,
                       bar(bars->kv_full[s]));
         }
-        ++issued;
       }
-      if (*abort_flag) {
-        // drain: wait (bounded) for the copies this thread issued that may still be landing
-        for (int g = 0; g < n_q; ++g) {
-          const unsigned long long t0 = global_timer();
-          while (!mbar_try(bar(bars->q_full[g]), 0) && global_timer() - t0 < kWaitLimitNs) {
-          }
+    }
+    if (*abort_flag) {
+      // drain: wait (bounded) for the copies this warp issued that may still be landing
+      if (seg_i > 0) {
+        const unsigned long long t0 = global_timer();
+        while (!mbar_try(bar(bars->q_full), (seg_i - 1) & 1) &&
+               global_timer() - t0 < kWaitLimitNs) {
         }
-        for (int j = max(0, issued - C::NS); j < issued; ++j) {
-          const unsigned long long t0 = global_timer();
-          while (!mbar_try(bar(bars->kv_full[j % C::NS]), (j / C::NS) & 1) &&
-                 global_timer() - t0 < kWaitLimitNs) {
-          }
+      }
+      for (int j = max(0, issued - C::NS); j < issued; ++j) {
+        const unsigned long long t0 = global_timer();
+        while (!mbar_try(bar(bars->kv_full[j % C::NS]), (j / C::NS) & 1) &&
+               global_timer() - t0 < kWaitLimitNs) {
         }
       }
     }
   } else if (warp == 1 || warp == 2) {
     // ---------------- MMA issuers: warp 1 for query tile 0, warp 2 for tile 1 ----------------
     const int g = warp - 1;
-    if (g < n_q) {  // whole warp, elected lane issues
-      constexpr uint32_t idesc_s = idesc_bf16(BM, BN, false);
-      constexpr uint32_t idesc_o = idesc_bf16(BM, D, true);
-      const uint32_t tS = tmem + 256 * g + TM::S;
-      const uint32_t tP = tmem + 256 * g + TM::P;
-      const uint32_t tO = tmem + 256 * g + TM::O;
-      const uint32_t q_base = sQ + g * C::TILE_BYTES;
-      bool ok = mbar_wait_warp(bar(bars->q_full[g]), 0, abort_flag, p.err, 2);
+    constexpr uint32_t idesc_s = idesc_bf16(BM, BN, false);
+    constexpr uint32_t idesc_o = idesc_bf16(BM, D, true);
+    const uint32_t tS = tmem + 256 * g + TM::S;
+    const uint32_t tP = tmem + 256 * g + TM::P;
+    const uint32_t tO = tmem + 256 * g + TM::O;
+    const uint32_t q_base = sQ + g * C::TILE_BYTES;
+    int ring = 0;     // key tiles consumed from the ring (all segments)
+    int jg = 0;       // key tiles processed by this query tile (all segments)
+    int segs = 0;     // segments this query tile took part in
+    int seg_i = 0;
+    bool ok = true;
+    for (long long x = lo; ok && x < hi; ++seg_i) {
+      const Segment sg = segment_at(p, x, hi, q_tiles);
+      x = (long long)sg.unit * p.n_tiles + sg.b;
+      const int n = sg.b - sg.a;
+      if (!mbar_wait_warp(bar(bars->q_full), seg_i & 1, abort_flag, p.err, 2)) {
+        ok = false;
+        break;
+      }
+      if (g >= sg.n_q) {
+        // no second query tile in this pair: release each ring stage and the query buffers
+        // after the tile has landed, so no arrival can run a phase ahead
+        for (int t = 0; t < n; ++t, ++ring) {
+          const int s = ring % C::NS;
+          if (!mbar_wait_warp(bar(bars->kv_full[s]), (ring / C::NS) & 1, abort_flag, p.err, 4)) {
+            ok = false;
+            break;
+          }
+          if (lane == 0) mbar_arrive(bar(bars->kv_empty[s]));
+        }
+        if (lane == 0) mbar_arrive(bar(bars->q_empty));
+        continue;
+      }
       tc_fence_after();
+      const int j0 = jg;  // first tile of this segment in this query tile's count
       auto issue_qk = [&](int j) -> bool {
-        const int s = j % C::NS;
-        if (!mbar_wait_warp(bar(bars->kv_full[s]), (j / C::NS) & 1, abort_flag, p.err, 4))
+        const int s = (ring + (j - j0)) % C::NS;
+        const int r = ring + (j - j0);
+        if (!mbar_wait_warp(bar(bars->kv_full[s]), (r / C::NS) & 1, abort_flag, p.err, 4))
           return false;
         if (j >= 1 && !mbar_wait_warp(bar(bars->s_free[g]), (j - 1) & 1, abort_flag, p.err, 5))
           return false;
@@ -458,21 +520,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       auto issue_pv = [&](int i) -> bool {
         if (!mbar_wait_warp(bar(bars->p_full[g]), i & 1, abort_flag, p.err, 3)) return false;
+        // O of the previous segment must have been read out before the first PV overwrites it
+        if (i == j0 && segs > 0 &&
+            !mbar_wait_warp(bar(bars->o_free[g]), (segs - 1) & 1, abort_flag, p.err, 13))
+          return false;
         tc_fence_after();
-        const int s = i % C::NS;
+        const int s = (ring + (i - j0)) % C::NS;
         const uint32_t v_base = sV + s * C::TILE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
           // B = V tile [keys][D], MN-major: 16 keys = 2 groups of 8 rows of 128 B
           const uint64_t bd = sdesc(v_base + kk * 2048, C::ATOM_BYTES, 1024);
-          mma_ts(tO, tP + 8 * kk, bd, idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(tO, tP + 8 * kk, bd, idesc_o, (i > j0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(bar(bars->pv_done[g]));
         mma_commit(bar(bars->kv_empty[s]));
         return true;
       };
-      if (ok && n > 0) ok = issue_qk(0);
-      for (int j = 1; ok && j < n; ++j) {
+      // with P written over S, the previous segment's last PV must have read P before the
+      // first S of this segment overwrites it
+      if (TM::kPAliasesS && j0 > 0)
+        ok = mbar_wait_warp(bar(bars->pv_done[g]), (j0 - 1) & 1, abort_flag, p.err, 14);
+      ok = ok && issue_qk(j0);
+      for (int j = j0 + 1; ok && j < j0 + n; ++j) {
         if (TM::kPAliasesS) {
           // P_{j-1} lives in S: PV_{j-1} must have read it before S_j overwrites it
           ok = issue_pv(j - 1) &&
@@ -483,128 +553,150 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = issue_qk(j) && issue_pv(j - 1);
         }
       }
-      if (ok && !*abort_flag && n > 0) issue_pv(n - 1);
-      // every MMA issued by this thread has completed once `drain` flips
-      mma_commit(bar(bars->drain[g]));
-      const unsigned long long t0 = global_timer();
-      while (!mbar_try(bar(bars->drain[g]), 0) && global_timer() - t0 < kWaitLimitNs) {
+      if (ok) {
+        // the last QK of the segment has been issued: the query buffers can be refilled once
+        // it completes
+        mma_commit(bar(bars->q_empty));
+        ok = issue_pv(j0 + n - 1);
       }
+      jg += n;
+      ring += n;
+      ++segs;
     }
-  }
-  } else {
+    // every MMA issued by this warp has completed once `drain` flips
+    mma_commit(bar(bars->drain[g]));
+    const unsigned long long t0 = global_timer();
+    while (!mbar_try(bar(bars->drain[g]), 0) && global_timer() - t0 < kWaitLimitNs) {
+    }
+  } else if (warp >= 4) {
     // ---------------- softmax + epilogue: warps 4..7 tile 0, warps 8..11 tile 1 ----------------
     const int g = (warp - 4) >> 2;
     const int quad = warp & 3;                  // TMEM lane quadrant this warp may access
-    const int row = (tile0 + g) * BM + quad * 32 + lane;
+    const int row_in_pair = g * BM + quad * 32 + lane;
     const uint32_t lane_base = tmem + 256 * g + ((uint32_t)(quad * 32) << 16);
     const uint32_t tS = lane_base + TM::S;
     const uint32_t tP = lane_base + TM::P;
     const uint32_t tO = lane_base + TM::O;
-    float m = -INFINITY;  // running max (log2 domain) the P values and O are relative to
-    float l = 0.f;
-    bool ok = g < n_q;
+    int jg = 0;
+    int seg_i = 0;
+    bool ok = true;
     uint32_t S[BN];
-    for (int j = 0; ok && j < n; ++j) {
-      // every wait in these warps is made warp-uniform, so warp-collective tcgen05 ops and
-      // votes below always run with the whole warp
-      if (!__all_sync(kFull, mbar_wait(bar(bars->s_full[g]), j & 1, abort_flag, p.err, 6))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
+    for (long long x = lo; ok && x < hi; ++seg_i) {
+      const Segment sg = segment_at(p, x, hi, q_tiles);
+      x = (long long)sg.unit * p.n_tiles + sg.b;
+      if (g >= sg.n_q) continue;
+      const int n = sg.b - sg.a;
+      const int j0 = jg;
+      float m = -INFINITY;  // running max (log2 domain) the P values and O are relative to
+      float l = 0.f;
+      for (int j = j0; ok && j < j0 + n; ++j) {
+        // every wait in these warps is made warp-uniform, so warp-collective tcgen05 ops and
+        // votes below always run with the whole warp
+        if (!__all_sync(kFull, mbar_wait(bar(bars->s_full[g]), j & 1, abort_flag, p.err, 6))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < BN / 32; ++c) tmem_ld32(tS + 32 * c, S + 32 * c);
-      tmem_wait_ld();
-      reg_fence<BN>(S);
-      tc_fence_before();
-      mbar_arrive(bar(bars->s_free[g]));
+        for (int c = 0; c < BN / 32; ++c) tmem_ld32(tS + 32 * c, S + 32 * c);
+        tmem_wait_ld();
+        reg_fence<BN>(S);
+        tc_fence_before();
+        mbar_arrive(bar(bars->s_free[g]));
 
-      const int valid = tile_ref(p, t_begin + j).valid;
-      if (valid != BN) {
-        // keys past the end of a page / of the special stream: -inf scores, zero weight
+        const int valid = tile_ref(p, sg.a + (j - j0)).valid;
+        if (valid != BN) {
+          // keys past the end of a page / of the special stream: -inf scores, zero weight
 #pragma unroll
-        for (int i = 0; i < BN; ++i)
-          if (i >= valid) S[i] = 0xff800000u;
+          for (int i = 0; i < BN; ++i)
+            if (i >= valid) S[i] = 0xff800000u;
+        }
+        float mx8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          mx8[i] = fmaxf(__uint_as_float(S[2 * i]), __uint_as_float(S[2 * i + 1]));
+#pragma unroll
+        for (int i = 16; i < BN; i += 2)
+          mx8[(i >> 1) & 7] = max3f(mx8[(i >> 1) & 7], __uint_as_float(S[i]),
+                                    __uint_as_float(S[i + 1]));
+        const float mx = max3f(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]),
+                               fmaxf(mx8[6], mx8[7]));
+        const float m_tile = mx * p.scale_log2;
+        bool rescale = false;
+        float alpha = 1.f;
+        if (m_tile > m + kRescaleThreshold) {
+          alpha = fast_exp2(m - m_tile);  // 0 on the first tile (m = -inf)
+          m = m_tile;
+          l *= alpha;
+          rescale = true;
+        }
+        // P_j overwrites P_{j-1} (and O may be rescaled): PV_{j-1} must have finished
+        if (j >= 1 && !__all_sync(kFull, mbar_wait(bar(bars->pv_done[g]), (j - 1) & 1,
+                                                   abort_flag, p.err, 7))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t c2 = pack_f2(p.scale_log2, p.scale_log2);
+        const uint64_t nm2 = pack_f2(-m, -m);
+        uint64_t l4[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int i0 = 32 * c + 2 * i;
+            float x0, x1;
+            unpack_f2(ffma2(pack_f2(__uint_as_float(S[i0]), __uint_as_float(S[i0 + 1])), c2,
+                            nm2),
+                      x0, x1);
+            const float p0 = fast_exp2(x0);
+            const float p1 = fast_exp2(x1);
+            l4[i & 3] = fadd2(l4[i & 3], pack_f2(p0, p1));
+            pk[i] = pack_bf16(p0, p1);
+          }
+          tmem_st16(tP + 16 * c, pk);
+        }
+        {
+          float a0, a1, b0, b1, c0, c1, d0, d1;
+          unpack_f2(l4[0], a0, a1);
+          unpack_f2(l4[1], b0, b1);
+          unpack_f2(l4[2], c0, c1);
+          unpack_f2(l4[3], d0, d1);
+          l += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
+        }
+        if (__any_sync(kFull, rescale) && j > j0) {
+          // O holds sum_{i<j} P_i V_i relative to the old max: scale it before PV_j lands
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tO + 32 * c, o);
+            tmem_wait_ld();
+            reg_fence<32>(o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st16(tO + 32 * c, o);
+            tmem_st16(tO + 32 * c + 16, o + 16);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(bars->p_full[g]));
       }
-      float mx8[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        mx8[i] = fmaxf(__uint_as_float(S[2 * i]), __uint_as_float(S[2 * i + 1]));
-#pragma unroll
-      for (int i = 16; i < BN; i += 2)
-        mx8[(i >> 1) & 7] = max3f(mx8[(i >> 1) & 7], __uint_as_float(S[i]),
-                                  __uint_as_float(S[i + 1]));
-      const float mx = max3f(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]),
-                             fmaxf(mx8[6], mx8[7]));
-      const float m_tile = mx * p.scale_log2;
-      bool rescale = false;
-      float alpha = 1.f;
-      if (m_tile > m + kRescaleThreshold) {
-        alpha = fast_exp2(m - m_tile);  // 0 on the first tile (m = -inf)
-        m = m_tile;
-        l *= alpha;
-        rescale = true;
-      }
-      // P_j overwrites P_{j-1} (and O may be rescaled): PV_{j-1} must have finished
-      if (j >= 1 && !__all_sync(kFull, mbar_wait(bar(bars->pv_done[g]), (j - 1) & 1,
-                                                 abort_flag, p.err, 7))) {
+      jg += n;
+      if (!ok ||
+          !__all_sync(kFull, mbar_wait(bar(bars->pv_done[g]), (jg - 1) & 1, abort_flag, p.err,
+                                       9))) {
         ok = false;
         break;
       }
-      tc_fence_after();
-      const uint64_t c2 = pack_f2(p.scale_log2, p.scale_log2);
-      const uint64_t nm2 = pack_f2(-m, -m);
-      uint64_t l4[4] = {0, 0, 0, 0};
-#pragma unroll
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int i0 = 32 * c + 2 * i;
-          float x0, x1;
-          unpack_f2(ffma2(pack_f2(__uint_as_float(S[i0]), __uint_as_float(S[i0 + 1])), c2, nm2),
-                    x0, x1);
-          const float p0 = fast_exp2(x0);
-          const float p1 = fast_exp2(x1);
-          l4[i & 3] = fadd2(l4[i & 3], pack_f2(p0, p1));
-          pk[i] = pack_bf16(p0, p1);
-        }
-        tmem_st16(tP + 16 * c, pk);
-      }
-      {
-        float a0, a1, b0, b1, c0, c1, d0, d1;
-        unpack_f2(l4[0], a0, a1);
-        unpack_f2(l4[1], b0, b1);
-        unpack_f2(l4[2], c0, c1);
-        unpack_f2(l4[3], d0, d1);
-        l += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
-      }
-      if (__any_sync(kFull, rescale) && j > 0) {
-        // O holds sum_{i<j} P_i V_i relative to the old max: scale it before PV_j lands
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + 32 * c, o);
-          tmem_wait_ld();
-          reg_fence<32>(o);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st16(tO + 32 * c, o);
-          tmem_st16(tO + 32 * c + 16, o + 16);
-        }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(bars->p_full[g]));
-    }
-    if (ok && n > 0 &&
-        __all_sync(kFull, mbar_wait(bar(bars->pv_done[g]), (n - 1) & 1, abort_flag, p.err, 9))) {
       tc_fence_after();
       const float inv_l = 1.f / l;
+      const int row = (2 * sg.pair) * BM + row_in_pair;
       const bool store = row < p.tokens;
-      if (p.n_splits == 1) {
+      if (sg.whole) {
         __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) +
-                             ((long long)row * p.heads + head) * D;
+                             ((long long)row * p.heads + sg.head) * D;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
@@ -624,7 +716,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       } else {
-        const long long r = ((long long)split * p.tokens + row) * p.heads + head;
+        // slot unit + c: one per (CTA, unit it touches), dense over CTAs in order
+        const long long slot = (long long)sg.unit + blockIdx.x;
+        const long long r = slot * (2 * BM) + row_in_pair;
         float* po = p.part_o + r * D;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
@@ -644,6 +738,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (store) p.part_lse[r] = m + __log2f(l);
       }
+      // O of this segment has been read: the next segment's first PV may overwrite it
+      tc_fence_before();
+      mbar_arrive(bar(bars->o_free[g]));
     }
   }
 
@@ -658,30 +755,49 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// Merges the partial results of the units that span more than one CTA:
 // out[row][h] = sum_s w_s o_s / sum_s w_s with w_s = 2^(lse_s - max_s lse_s).
-// One warp per (row, head); lane d covers features d, d+32, ... .
+// One warp per (unit, row of the pair); lane d covers features d, d+32, ...
 template <int D>
-__global__ void __launch_bounds__(256)
-    attn_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
-                        __nv_bfloat16* __restrict__ out, int n_splits, int rows_total) {
-  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+__global__ void __launch_bounds__(256) attn_combine_kernel(const __grid_constant__ AttnParams p) {
+  const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  if (gw >= rows_total) return;
+  const long long units = (long long)p.n_pairs * p.heads;
+  if (gw >= units * (2 * BM)) return;
+  const int unit = (int)(gw / (2 * BM));
+  const int row_in_pair = (int)(gw - (long long)unit * (2 * BM));
+  const int pair = unit % p.n_pairs;
+  const int head = unit / p.n_pairs;
+  const int row = 2 * pair * BM + row_in_pair;
+  if (row >= p.tokens) return;
+  const long long first = (long long)unit * p.n_tiles;
+  const long long last = first + p.n_tiles - 1;
+  // CTAs whose share [sk_lo(c), sk_lo(c+1)) meets this unit
+  int c0 = (int)(first * p.grid / p.work);
+  while (c0 > 0 && sk_lo(p.work, p.grid, c0) > first) --c0;
+  while (sk_lo(p.work, p.grid, c0 + 1) <= first) ++c0;
+  int c1 = c0;
+  while (c1 + 1 < p.grid && sk_lo(p.work, p.grid, c1 + 1) <= last) ++c1;
+  if (c1 == c0) return;  // one CTA did the whole unit and wrote the output itself
   float mx = -INFINITY;
-  for (int s = 0; s < n_splits; ++s) mx = fmaxf(mx, part_lse[(long long)s * rows_total + gw]);
+  for (int c = c0; c <= c1; ++c) {
+    const long long r = ((long long)unit + c) * (2 * BM) + row_in_pair;
+    mx = fmaxf(mx, p.part_lse[r]);
+  }
   float acc[D / 32];
 #pragma unroll
   for (int i = 0; i < D / 32; ++i) acc[i] = 0.f;
   float wsum = 0.f;
-  for (int s = 0; s < n_splits; ++s) {
-    const float w = exp2f(part_lse[(long long)s * rows_total + gw] - mx);
+  for (int c = c0; c <= c1; ++c) {
+    const long long r = ((long long)unit + c) * (2 * BM) + row_in_pair;
+    const float w = exp2f(p.part_lse[r] - mx);
     wsum += w;
-    const float* po = part_o + ((long long)s * rows_total + gw) * D;
+    const float* po = p.part_o + r * D;
 #pragma unroll
     for (int i = 0; i < D / 32; ++i) acc[i] = fmaf(w, po[lane + 32 * i], acc[i]);
   }
   const float inv = 1.f / wsum;
-  __nv_bfloat16* o = out + (long long)gw * D;
+  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + ((long long)row * p.heads + head) * D;
 #pragma unroll
   for (int i = 0; i < D / 32; ++i) o[lane + 32 * i] = __float2bfloat16_rn(acc[i] * inv);
 }
@@ -705,8 +821,8 @@ cudaError_t prepare_attn_tc() {
 
 }  // namespace
 
-cudaError_t launch_attn_tc(const AttnParams& p, int head_dim, int q_tiles, cudaStream_t s) {
-  dim3 grid((q_tiles + 1) / 2, p.n_splits, p.heads);
+cudaError_t launch_attn_tc(const AttnParams& p, int head_dim, cudaStream_t s) {
+  const dim3 grid(p.grid);
   cudaError_t e;
   if (head_dim == 64) {
     if ((e = prepare_attn_tc<64>()) != cudaSuccess) return e;
@@ -720,19 +836,13 @@ cudaError_t launch_attn_tc(const AttnParams& p, int head_dim, int q_tiles, cudaS
   return cudaGetLastError();
 }
 
-cudaError_t launch_attn_combine(const float* part_o, const float* part_lse, void* out,
-                                int n_splits, int tokens, int heads, int head_dim,
-                                cudaStream_t s) {
-  const int rows = tokens * heads;
-  const int blocks = (rows * 32 + 255) / 256;
+cudaError_t launch_attn_combine(const AttnParams& p, int head_dim, cudaStream_t s) {
+  const long long warps = (long long)p.n_pairs * p.heads * (2 * BM);
+  const unsigned blocks = (unsigned)((warps * 32 + 255) / 256);
   if (head_dim == 64)
-    attn_combine_kernel<64><<<blocks, 256, 0, s>>>(part_o, part_lse,
-                                                   static_cast<__nv_bfloat16*>(out), n_splits,
-                                                   rows);
+    attn_combine_kernel<64><<<blocks, 256, 0, s>>>(p);
   else if (head_dim == 128)
-    attn_combine_kernel<128><<<blocks, 256, 0, s>>>(part_o, part_lse,
-                                                    static_cast<__nv_bfloat16*>(out), n_splits,
-                                                    rows);
+    attn_combine_kernel<128><<<blocks, 256, 0, s>>>(p);
   else
     return cudaErrorInvalidValue;
   return cudaGetLastError();

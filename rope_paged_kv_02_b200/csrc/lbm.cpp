@@ -30,10 +30,10 @@ struct lbm_cache {
   const lbm_rope* rope = nullptr;
   lbm::Pools pools{};
   void* pool_mem = nullptr;     // one allocation holding the four pools
-  float* part_o = nullptr;      // split-KV partial outputs
+  float* part_o = nullptr;      // partial outputs of units shared by several CTAs
   float* part_lse = nullptr;
-  int max_splits = 1;
-  int forced_splits = 0;        // LBM_ATTN_SPLITS at create time (0: planned per frame)
+  size_t scratch_floats = 0;    // capacity of part_o + part_lse in floats
+  int forced_grid = 0;          // LBM_ATTN_GRID at create time (0: one CTA per SM)
   int* d_err = nullptr;
   long long device_bytes = 0;
   long long launches = 0;       // kernels launched so far
@@ -49,7 +49,6 @@ struct lbm_cache {
 
 namespace {
 
-constexpr int kMaxSplits = 16;
 constexpr int kKeyTile = 128;  // keys per attention key tile (page strides are multiples)
 
 int elem_size(int dtype) { return dtype == LBM_BF16 ? 2 : 4; }
@@ -103,26 +102,43 @@ void order_after(lbm_cache* c, cudaStream_t s) {
   c->ev_valid = true;
 }
 
-// Number of key splits: minimise waves x (tiles per split + fixed cost) + combine cost.
-int plan_splits(int work_units, int n_tiles, int num_sms, double combine_tiles_per_split,
-                int max_splits) {
-  int best = 1;
-  double best_cost = 1e30;
-  const int lim = n_tiles < max_splits ? n_tiles : max_splits;
-  for (int s = 1; s <= lim; ++s) {
-    const int tps = (n_tiles + s - 1) / s;
-    const int s_eff = (n_tiles + tps - 1) / tps;
-    if (s_eff != s) continue;
-    const long long units = (long long)work_units * s;
-    const long long waves = (units + num_sms - 1) / num_sms;
-    double cost = (double)waves * (tps + 4.0);
-    if (s > 1) cost += 8.0 + combine_tiles_per_split * s;
-    if (cost < best_cost - 1e-9) {
-      best_cost = cost;
-      best = s;
-    }
+// Fills everything of the attention parameters but the partial-result scratch: the visible
+// page list (no container), tensor maps, and the stream-K partition of the frame's work
+// over the persistent CTAs.  Returns LBM_OK or an error status.
+int fill_attn_params(lbm_cache* c, const void* q, void* out, lbm::AttnParams& p) {
+  int n_pages = 0;
+  for (const auto& e : c->pager.scale()) p.pages[n_pages++] = (uint16_t)e.page;
+  for (const auto& e : c->pager.window()) p.pages[n_pages++] = (uint16_t)e.page;
+  p.pages[n_pages++] = (uint16_t)c->pager.pending_page();
+  const int n_sp = c->pager.n_special() + c->psi;
+  const int T = c->psi + c->patches;
+  if (q != c->tm_q_ptr) {
+    const uint64_t row = (uint64_t)c->head_dim * 2;
+    if (!make_map(&c->tm_q, q, c->head_dim, c->heads, T, row, row * c->heads, 1, 128))
+      return LBM_ERR_CUDA;
+    c->tm_q_ptr = q;
   }
-  return best;
+  p.tm_q = c->tm_q;
+  p.tm_kp = c->tm_kp;
+  p.tm_vp = c->tm_vp;
+  p.tm_ks = c->tm_ks;
+  p.tm_vs = c->tm_vs;
+  p.out = out;
+  p.err = c->d_err;
+  p.tokens = T;
+  p.heads = c->heads;
+  p.patches = c->patches;
+  p.page_stride = c->pools.page_stride;
+  p.tiles_per_page = (c->patches + kKeyTile - 1) / kKeyTile;
+  p.n_pages = n_pages;
+  p.n_special = n_sp;
+  p.n_tiles = p.n_pages * p.tiles_per_page + (n_sp + kKeyTile - 1) / kKeyTile;
+  p.n_pairs = ((T + 127) / 128 + 1) / 2;
+  p.work = (long long)p.n_pairs * c->heads * p.n_tiles;
+  const long long want = c->forced_grid ? c->forced_grid : c->num_sms;
+  p.grid = (int)std::min<long long>(want, p.work);
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)c->head_dim));
+  return LBM_OK;
 }
 
 }  // namespace
@@ -242,9 +258,9 @@ int lbm_cache_create(int heads, int head_dim, int patches_per_frame, int special
   c->rope = rope;
   cudaGetDevice(&c->device);
   cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device);
-  if (const char* env = std::getenv("LBM_ATTN_SPLITS")) {
+  if (const char* env = std::getenv("LBM_ATTN_GRID")) {
     const int v = std::atoi(env);
-    if (v >= 1 && v <= kMaxSplits) c->forced_splits = v;
+    if (v >= 1 && v <= 4 * c->num_sms) c->forced_grid = v;
   }
 
   const int P = scale_frames + sliding_window + 1;
@@ -255,9 +271,12 @@ int lbm_cache_create(int heads, int head_dim, int patches_per_frame, int special
   const size_t spec_bytes = (size_t)heads * cap * head_dim * e;
   const size_t total = 2 * patch_bytes + 2 * spec_bytes;
   const int T = specials_per_frame + patches_per_frame;
-  c->max_splits = dtype == LBM_BF16 ? kMaxSplits : 1;
-  const size_t part_o_bytes = (size_t)c->max_splits * T * heads * head_dim * sizeof(float);
-  const size_t part_lse_bytes = (size_t)c->max_splits * T * heads * sizeof(float);
+  // partial results: (units + persistent CTAs) slots of 256 rows x (head_dim + 1) floats
+  const long long units = (long long)(((T + 127) / 128 + 1) / 2) * heads;
+  const int grid_max = c->forced_grid ? c->forced_grid : c->num_sms;
+  c->scratch_floats = lbm::sk_scratch_floats(units, grid_max, head_dim);
+  const size_t part_o_bytes = (size_t)(units + grid_max) * 256 * head_dim * sizeof(float);
+  const size_t part_lse_bytes = (size_t)(units + grid_max) * 256 * sizeof(float);
   auto fail = [&](int st) {
     cudaFree(c->pool_mem);
     cudaFree(c->part_o);
@@ -350,45 +369,17 @@ int lbm_attend_frame(lbm_cache_t* c, const void* q, void* out, void* stream) {
   order_before(c, s);
   if (c->dtype == LBM_BF16) {
     static thread_local lbm::AttnParams p;  // ~3 KB: kept off the stack
-    if (q != c->tm_q_ptr) {
-      const uint64_t row = (uint64_t)c->head_dim * 2;
-      if (!make_map(&c->tm_q, q, c->head_dim, c->heads, T, row, row * c->heads, 1, 128))
-        return LBM_ERR_CUDA;
-      c->tm_q_ptr = q;
-    }
-    p.tm_q = c->tm_q;
-    p.tm_kp = c->tm_kp;
-    p.tm_vp = c->tm_vp;
-    p.tm_ks = c->tm_ks;
-    p.tm_vs = c->tm_vs;
-    p.out = out;
-    p.part_o = c->part_o;
+    const int st = fill_attn_params(c, q, out, p);
+    if (st != LBM_OK) return st;
+    const long long units = (long long)p.n_pairs * c->heads;
+    if (lbm::sk_scratch_floats(units, p.grid, c->head_dim) > c->scratch_floats)
+      return LBM_ERR_CAPACITY;
+    p.part_o = c->part_o;      // sized for (units + max grid) slots at creation
     p.part_lse = c->part_lse;
-    p.err = c->d_err;
-    p.tokens = T;
-    p.heads = c->heads;
-    p.patches = c->patches;
-    p.page_stride = c->pools.page_stride;
-    p.tiles_per_page = (c->patches + kKeyTile - 1) / kKeyTile;
-    p.n_pages = (int)pages.size();
-    p.n_special = n_sp;
-    p.n_tiles = p.n_pages * p.tiles_per_page + (n_sp + kKeyTile - 1) / kKeyTile;
-    p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)c->head_dim));
-    for (size_t i = 0; i < pages.size(); ++i) p.pages[i] = (uint16_t)pages[i];
-    const int q_tiles = (T + 127) / 128;
-    // combine cost of one split, in key-tile times (a tile of both query tiles ~1 us)
-    const double combine = (double)T * c->heads * c->head_dim * 4.0 / 6.0e6;
-    p.n_splits = plan_splits((q_tiles + 1) / 2 * c->heads, p.n_tiles, c->num_sms, combine,
-                             c->max_splits);
-    if (c->forced_splits) p.n_splits = std::min(c->forced_splits, p.n_tiles);
-    p.tiles_per_split = (p.n_tiles + p.n_splits - 1) / p.n_splits;
-    p.n_splits = (p.n_tiles + p.tiles_per_split - 1) / p.tiles_per_split;  // no empty split
-    if (lbm::launch_attn_tc(p, c->head_dim, q_tiles, s) != cudaSuccess) return LBM_ERR_CUDA;
+    if (lbm::launch_attn_tc(p, c->head_dim, s) != cudaSuccess) return LBM_ERR_CUDA;
     ++c->launches;
-    if (p.n_splits > 1) {
-      if (lbm::launch_attn_combine(c->part_o, c->part_lse, out, p.n_splits, T, c->heads,
-                                   c->head_dim, s) != cudaSuccess)
-        return LBM_ERR_CUDA;
+    if (lbm::sk_has_split(p.work, p.grid, p.n_tiles)) {
+      if (lbm::launch_attn_combine(p, c->head_dim, s) != cudaSuccess) return LBM_ERR_CUDA;
       ++c->launches;
     }
   } else {
@@ -429,54 +420,20 @@ int lbm_attend_frame_noalloc(lbm_cache_t* c, const void* q, void* out, void* str
   const int st = lbm::noalloc_scratch(c->device, &scratch, &scratch_floats);
   if (st != LBM_OK) return st;
   lbm::AttnParams p;  // on the stack: this call touches no heap
-  // visible pages in page-table order, built without a container
-  int n_pages = 0;
-  for (const auto& e : c->pager.scale()) p.pages[n_pages++] = (uint16_t)e.page;
-  for (const auto& e : c->pager.window()) p.pages[n_pages++] = (uint16_t)e.page;
-  p.pages[n_pages++] = (uint16_t)c->pager.pending_page();
-  const int n_sp = c->pager.n_special() + c->psi;
-  const int T = c->psi + c->patches;
-  const uint64_t row = (uint64_t)c->head_dim * 2;
-  if (q != c->tm_q_ptr) {
-    if (!make_map(&c->tm_q, q, c->head_dim, c->heads, T, row, row * c->heads, 1, 128))
-      return LBM_ERR_CUDA;
-    c->tm_q_ptr = q;
-  }
-  p.tm_q = c->tm_q;
-  p.tm_kp = c->tm_kp;
-  p.tm_vp = c->tm_vp;
-  p.tm_ks = c->tm_ks;
-  p.tm_vs = c->tm_vs;
-  p.out = out;
-  p.err = c->d_err;
-  p.tokens = T;
-  p.heads = c->heads;
-  p.patches = c->patches;
-  p.page_stride = c->pools.page_stride;
-  p.tiles_per_page = (c->patches + kKeyTile - 1) / kKeyTile;
-  p.n_pages = n_pages;
-  p.n_special = n_sp;
-  p.n_tiles = p.n_pages * p.tiles_per_page + (n_sp + kKeyTile - 1) / kKeyTile;
-  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)c->head_dim));
-  const int q_tiles = (T + 127) / 128;
-  const double combine = (double)T * c->heads * c->head_dim * 4.0 / 6.0e6;
-  p.n_splits = plan_splits((q_tiles + 1) / 2 * c->heads, p.n_tiles, c->num_sms, combine,
-                           c->max_splits);
-  if (c->forced_splits) p.n_splits = std::min(c->forced_splits, p.n_tiles);
-  p.tiles_per_split = (p.n_tiles + p.n_splits - 1) / p.n_splits;
-  p.n_splits = (p.n_tiles + p.tiles_per_split - 1) / p.tiles_per_split;
-  const size_t rows = (size_t)p.n_splits * T * c->heads;
-  if (p.n_splits > 1 && rows * (c->head_dim + 1) > scratch_floats) return LBM_ERR_CAPACITY;
+  const int pst = fill_attn_params(c, q, out, p);
+  if (pst != LBM_OK) return pst;
+  const long long units = (long long)p.n_pairs * c->heads;
+  const bool split = lbm::sk_has_split(p.work, p.grid, p.n_tiles);
+  if (split && lbm::sk_scratch_floats(units, p.grid, c->head_dim) > scratch_floats)
+    return LBM_ERR_CAPACITY;
   p.part_o = scratch;
-  p.part_lse = scratch + rows * c->head_dim;
+  p.part_lse = scratch + (size_t)(units + p.grid) * 256 * c->head_dim;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   order_before(c, s);
-  if (lbm::launch_attn_tc(p, c->head_dim, q_tiles, s) != cudaSuccess) return LBM_ERR_CUDA;
+  if (lbm::launch_attn_tc(p, c->head_dim, s) != cudaSuccess) return LBM_ERR_CUDA;
   ++c->launches;
-  if (p.n_splits > 1) {
-    if (lbm::launch_attn_combine(p.part_o, p.part_lse, out, p.n_splits, T, c->heads,
-                                 c->head_dim, s) != cudaSuccess)
-      return LBM_ERR_CUDA;
+  if (split) {
+    if (lbm::launch_attn_combine(p, c->head_dim, s) != cudaSuccess) return LBM_ERR_CUDA;
     ++c->launches;
   }
   order_after(c, s);

@@ -44,6 +44,16 @@ struct AppendArgs {
 constexpr int kMaxPages = 1024;
 
 // Kernel parameter block of the paged attention (passed by value).
+// Stream-K partition of one frame's attention over `grid` persistent CTAs.  A unit is one
+// (pair of 128-row query tiles, head), unit u = head * n_pairs + pair; its key tiles are the
+// global work items [u * n_tiles, (u + 1) * n_tiles).  CTA c processes the contiguous items
+// [sk_lo(c), sk_lo(c + 1)), i.e. a run of segments (unit, key-tile range); a segment that
+// is a whole unit writes the final output, any other writes a partial (O, LSE) into slot
+// unit + c (dense: at most units + grid slots), merged by the combine kernel.
+__host__ __device__ inline long long sk_lo(long long work, int grid, int c) {
+  return (long long)c * work / grid;
+}
+
 struct AttnParams {
   CUtensorMap tm_q;      // q   {head_dim, heads, T}
   CUtensorMap tm_kp;     // K patch pool {head_dim, P*stride, heads}
@@ -51,8 +61,8 @@ struct AttnParams {
   CUtensorMap tm_ks;     // K special pool {head_dim, spec_cap, heads}
   CUtensorMap tm_vs;
   void* out;             // [T][heads][head_dim] bf16
-  float* part_o;         // [splits][T][heads][head_dim] fp32 (split mode)
-  float* part_lse;       // [splits][T][heads] log2-domain LSE (split mode)
+  float* part_o;         // [units + grid slots][256 rows][head_dim] fp32 partial outputs
+  float* part_lse;       // [units + grid slots][256 rows] log2-domain LSE
   int* err;              // device error word (bounded waits)
   int tokens;            // T
   int heads;
@@ -62,8 +72,9 @@ struct AttnParams {
   int n_pages;           // visible patch pages
   int n_special;         // visible special tokens
   int n_tiles;           // n_pages * tiles_per_page + ceil(n_special / 128)
-  int tiles_per_split;
-  int n_splits;
+  int n_pairs;           // ceil(ceil(T / 128) / 2) query-tile pairs
+  long long work;        // n_pairs * heads * n_tiles
+  int grid;              // persistent CTAs
   float scale_log2;      // log2(e) / sqrt(head_dim)
   uint16_t pages[kMaxPages];
 };
@@ -90,10 +101,19 @@ cudaError_t launch_rope_append(const RopeTables& rt, const Pools& pools,
 
 // attn_tc.cu (bf16, tcgen05)
 size_t attn_tc_smem_bytes(int head_dim);
-cudaError_t launch_attn_tc(const AttnParams& p, int head_dim, int q_tiles, cudaStream_t s);
-cudaError_t launch_attn_combine(const float* part_o, const float* part_lse, void* out,
-                                int n_splits, int tokens, int heads, int head_dim,
-                                cudaStream_t s);
+cudaError_t launch_attn_tc(const AttnParams& p, int head_dim, cudaStream_t s);
+// merges the partial results of every unit that spans more than one CTA
+cudaError_t launch_attn_combine(const AttnParams& p, int head_dim, cudaStream_t s);
+// floats of partial results a frame may write: (units + grid) slots of 256 rows x (D + 1)
+inline size_t sk_scratch_floats(long long units, int grid, int head_dim) {
+  return (size_t)(units + grid) * 256 * (size_t)(head_dim + 1);
+}
+// true when some unit is shared by two CTAs (then the combine kernel must run)
+inline bool sk_has_split(long long work, int grid, int n_tiles) {
+  for (int c = 1; c < grid; ++c)
+    if (sk_lo(work, grid, c) % n_tiles != 0) return true;
+  return false;
+}
 
 // attn_static.cu: device address of the file-scope split-KV scratch on `device` (current)
 int noalloc_scratch(int device, float** ptr, size_t* floats);

@@ -69,9 +69,9 @@ def test_small_streams_all_frames_all_rows(cfg):
     run_stream(cfg)
 
 
-@pytest.mark.parametrize("splits", ["1", "3", "16"])
-def test_forced_split_counts_agree(splits, monkeypatch):
-    monkeypatch.setenv("LBM_ATTN_SPLITS", splits)
+@pytest.mark.parametrize("grid", ["1", "3", "16", "148"])
+def test_forced_grid_sizes_agree(grid, monkeypatch):
+    monkeypatch.setenv("LBM_ATTN_GRID", grid)
     run_stream(custom_config(205, 2, 64, "bf16", 12, 12, 8, 1, 2, 3))
 
 
