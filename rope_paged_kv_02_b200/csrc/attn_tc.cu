@@ -330,23 +330,25 @@ struct TmemMap {
 
 // One run of key tiles of one unit, as a CTA walks its share of the work.
 struct Segment {
-  int unit, pair, head, a, b;   // key tiles [a, b) of unit (pair, head)
-  int n_q;                      // query tiles of the pair (1 for an odd last pair)
-  bool whole;                   // the segment is the whole unit: write the final output
+  int unit, a, b;   // key tiles [a, b) of the unit
 };
 
-__device__ __forceinline__ Segment segment_at(const AttnParams& p, long long x, long long hi,
-                                              int q_tiles) {
+// Work items are counted in 32-bit integers: the host keeps a frame's work below 2^31.
+__device__ __forceinline__ Segment segment_at(const AttnParams& p, int x, int hi) {
   Segment sg;
-  sg.unit = (int)(x / p.n_tiles);
-  sg.pair = sg.unit % p.n_pairs;
-  sg.head = sg.unit / p.n_pairs;
-  sg.a = (int)(x - (long long)sg.unit * p.n_tiles);
-  const long long end = min(hi, (long long)(sg.unit + 1) * p.n_tiles);
-  sg.b = (int)(end - (long long)sg.unit * p.n_tiles);
-  sg.n_q = min(2, q_tiles - 2 * sg.pair);
-  sg.whole = sg.a == 0 && sg.b == p.n_tiles;
+  sg.unit = x / p.n_tiles;
+  sg.a = x - sg.unit * p.n_tiles;
+  sg.b = min(hi, (sg.unit + 1) * p.n_tiles) - sg.unit * p.n_tiles;
   return sg;
+}
+__device__ __forceinline__ int seg_pair(const AttnParams& p, const Segment& sg) {
+  return sg.unit % p.n_pairs;
+}
+__device__ __forceinline__ int seg_head(const AttnParams& p, const Segment& sg) {
+  return sg.unit / p.n_pairs;
+}
+__device__ __forceinline__ int seg_nq(const AttnParams& p, const Segment& sg, int q_tiles) {
+  return min(2, q_tiles - 2 * seg_pair(p, sg));
 }
 
 // Persistent CTA c of p.grid walks the global work items [sk_lo(c), sk_lo(c+1)).  Every role
@@ -367,8 +369,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = __shfl_sync(0xffffffffu, (int)(threadIdx.x >> 5), 0);
   const int lane = threadIdx.x & 31;
   const int q_tiles = (p.tokens + BM - 1) / BM;
-  const long long lo = sk_lo(p.work, p.grid, blockIdx.x);
-  const long long hi = sk_lo(p.work, p.grid, blockIdx.x + 1);
+  const int lo = (int)sk_lo(p.work, p.grid, blockIdx.x);
+  const int hi = (int)sk_lo(p.work, p.grid, blockIdx.x + 1);
 
   const uint32_t sQ = smem_u32(smem + C::OFF_Q);
   const uint32_t sK = smem_u32(smem + C::OFF_K);
@@ -410,21 +412,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     int issued = 0;        // key tiles issued so far (ring position)
     int seg_i = 0;
     bool ok = true;
-    for (long long x = lo; ok && x < hi; ++seg_i) {
-      const Segment sg = segment_at(p, x, hi, q_tiles);
-      x = (long long)sg.unit * p.n_tiles + sg.b;
+    for (int x = lo; ok && x < hi; ++seg_i) {
+      const Segment sg = segment_at(p, x, hi);
+      x = sg.unit * p.n_tiles + sg.b;
       // the query buffers are free once both MMA issuers are done with the last segment
       if (seg_i > 0 &&
           !mbar_wait_warp(bar(bars->q_empty), (seg_i - 1) & 1, abort_flag, p.err, 12)) {
         ok = false;
         break;
       }
-      mbar_expect_tx(bar(bars->q_full), sg.n_q * C::TILE_BYTES);
-      for (int g = 0; g < sg.n_q; ++g) {
+      const int n_q = seg_nq(p, sg, q_tiles);
+      const int head = seg_head(p, sg);
+      mbar_expect_tx(bar(bars->q_full), n_q * C::TILE_BYTES);
+      for (int g = 0; g < n_q; ++g) {
 #pragma unroll
         for (int a = 0; a < C::ATOMS; ++a)
-          tma_load_3d(sQ + g * C::TILE_BYTES + a * C::ATOM_BYTES, &p.tm_q, 64 * a, sg.head,
-                      (2 * sg.pair + g) * BM, bar(bars->q_full));
+          tma_load_3d(sQ + g * C::TILE_BYTES + a * C::ATOM_BYTES, &p.tm_q, 64 * a, head,
+                      (2 * seg_pair(p, sg) + g) * BM, bar(bars->q_full));
       }
       for (int t = sg.a; t < sg.b; ++t, ++issued) {
         const int s = issued % C::NS;
@@ -440,9 +444,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_expect_tx(bar(bars->kv_full[s]), 2 * C::TILE_BYTES);
 #pragma unroll
         for (int a = 0; a < C::ATOMS; ++a) {
-          tma_load_3d(sK + s * C::TILE_BYTES + a * C::ATOM_BYTES, tk, 64 * a, tr.row0, sg.head,
+          tma_load_3d(sK + s * C::TILE_BYTES + a * C::ATOM_BYTES, tk, 64 * a, tr.row0, head,
                       bar(bars->kv_full[s]));
-          tma_load_3d(sV + s * C::TILE_BYTES + a * C::ATOM_BYTES, tv, 64 * a, tr.row0, sg.head,
+          tma_load_3d(sV + s * C::TILE_BYTES + a * C::ATOM_BYTES, tv, 64 * a, tr.row0, head,
                       bar(bars->kv_full[s]));
         }
       }
@@ -476,15 +480,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     int segs = 0;     // segments this query tile took part in
     int seg_i = 0;
     bool ok = true;
-    for (long long x = lo; ok && x < hi; ++seg_i) {
-      const Segment sg = segment_at(p, x, hi, q_tiles);
-      x = (long long)sg.unit * p.n_tiles + sg.b;
+    for (int x = lo; ok && x < hi; ++seg_i) {
+      const Segment sg = segment_at(p, x, hi);
+      x = sg.unit * p.n_tiles + sg.b;
       const int n = sg.b - sg.a;
       if (!mbar_wait_warp(bar(bars->q_full), seg_i & 1, abort_flag, p.err, 2)) {
         ok = false;
         break;
       }
-      if (g >= sg.n_q) {
+      if (g >= seg_nq(p, sg, q_tiles)) {
         // no second query tile in this pair: release each ring stage and the query buffers
         // after the tile has landed, so no arrival can run a phase ahead
         for (int t = 0; t < n; ++t, ++ring) {
@@ -581,10 +585,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     int seg_i = 0;
     bool ok = true;
     uint32_t S[BN];
-    for (long long x = lo; ok && x < hi; ++seg_i) {
-      const Segment sg = segment_at(p, x, hi, q_tiles);
-      x = (long long)sg.unit * p.n_tiles + sg.b;
-      if (g >= sg.n_q) continue;
+    for (int x = lo; ok && x < hi; ++seg_i) {
+      const Segment sg = segment_at(p, x, hi);
+      x = sg.unit * p.n_tiles + sg.b;
+      if (g >= seg_nq(p, sg, q_tiles)) continue;
       const int n = sg.b - sg.a;
       const int j0 = jg;
       float m = -INFINITY;  // running max (log2 domain) the P values and O are relative to
@@ -692,11 +696,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const float inv_l = 1.f / l;
-      const int row = (2 * sg.pair) * BM + row_in_pair;
+      const int row = (2 * seg_pair(p, sg)) * BM + row_in_pair;
       const bool store = row < p.tokens;
-      if (sg.whole) {
+      if (sg.a == 0 && sg.b == p.n_tiles) {   // the whole unit: write the final output
         __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) +
-                             ((long long)row * p.heads + sg.head) * D;
+                             ((long long)row * p.heads + seg_head(p, sg)) * D;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];

@@ -135,6 +135,7 @@ int fill_attn_params(lbm_cache* c, const void* q, void* out, lbm::AttnParams& p)
   p.n_tiles = p.n_pages * p.tiles_per_page + (n_sp + kKeyTile - 1) / kKeyTile;
   p.n_pairs = ((T + 127) / 128 + 1) / 2;
   p.work = (long long)p.n_pairs * c->heads * p.n_tiles;
+  if (p.work >= (1LL << 31)) return LBM_ERR_UNSUPPORTED;  // the kernel counts in 32 bits
   const long long want = c->forced_grid ? c->forced_grid : c->num_sms;
   p.grid = (int)std::min<long long>(want, p.work);
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)c->head_dim));
