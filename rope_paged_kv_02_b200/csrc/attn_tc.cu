@@ -406,6 +406,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = __shfl_sync(0xffffffffu, bars->tmem_base, 0);
+  // launched as a programmatic dependent of the append kernel: the set-up above overlapped
+  // its tail; the pages it writes are read only after it has finished
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (warp == 0) {
     // ---------------- TMA producer (whole warp, elected lane issues) ----------------
@@ -761,9 +764,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // Merges the partial results of the units that span more than one CTA:
 // out[row][h] = sum_s w_s o_s / sum_s w_s with w_s = 2^(lse_s - max_s lse_s).
-// One warp per (unit, row of the pair); lane d covers features d, d+32, ...
+// One warp per (unit, row of the pair).  Lane s loads the LSE of segment s (32 segments at a
+// time), the warp reduces max and weights with shuffles, then every lane loads its features
+// of all segments back to back, so the loads of a row overlap instead of chaining.
 template <int D>
 __global__ void __launch_bounds__(256) attn_combine_kernel(const __grid_constant__ AttnParams p) {
+  constexpr int VPL = D / 32;  // features per lane
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // partials of the attention kernel
   const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const long long units = (long long)p.n_pairs * p.heads;
@@ -776,34 +783,59 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const __grid_constant
   if (row >= p.tokens) return;
   const long long first = (long long)unit * p.n_tiles;
   const long long last = first + p.n_tiles - 1;
-  // CTAs whose share [sk_lo(c), sk_lo(c+1)) meets this unit
+  // CTAs whose share [sk_lo(c), sk_lo(c+1)) meets this unit: c0 .. c1
   int c0 = (int)(first * p.grid / p.work);
   while (c0 > 0 && sk_lo(p.work, p.grid, c0) > first) --c0;
   while (sk_lo(p.work, p.grid, c0 + 1) <= first) ++c0;
-  int c1 = c0;
+  int c1 = (int)(last * p.grid / p.work);
   while (c1 + 1 < p.grid && sk_lo(p.work, p.grid, c1 + 1) <= last) ++c1;
+  while (c1 > c0 && sk_lo(p.work, p.grid, c1) > last) --c1;
   if (c1 == c0) return;  // one CTA did the whole unit and wrote the output itself
+  const int nseg = c1 - c0 + 1;
+  // partial row of segment (CTA c0 + s): slot unit + c
+  auto prow = [&](int s) { return ((long long)unit + c0 + s) * (2 * BM) + row_in_pair; };
   float mx = -INFINITY;
-  for (int c = c0; c <= c1; ++c) {
-    const long long r = ((long long)unit + c) * (2 * BM) + row_in_pair;
-    mx = fmaxf(mx, p.part_lse[r]);
+  for (int s0 = 0; s0 < nseg; s0 += 32) {
+    const float v = s0 + lane < nseg ? p.part_lse[prow(s0 + lane)] : -INFINITY;
+    mx = fmaxf(mx, v);
   }
-  float acc[D / 32];
 #pragma unroll
-  for (int i = 0; i < D / 32; ++i) acc[i] = 0.f;
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  float acc[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) acc[i] = 0.f;
   float wsum = 0.f;
-  for (int c = c0; c <= c1; ++c) {
-    const long long r = ((long long)unit + c) * (2 * BM) + row_in_pair;
-    const float w = exp2f(p.part_lse[r] - mx);
-    wsum += w;
-    const float* po = p.part_o + r * D;
-#pragma unroll
-    for (int i = 0; i < D / 32; ++i) acc[i] = fmaf(w, po[lane + 32 * i], acc[i]);
+  for (int s0 = 0; s0 < nseg; s0 += 32) {
+    const float w_lane =
+        s0 + lane < nseg ? exp2f(p.part_lse[prow(s0 + lane)] - mx) : 0.f;
+    const int cnt = min(32, nseg - s0);
+    for (int k = 0; k < cnt; ++k) {
+      const float w = __shfl_sync(0xffffffffu, w_lane, k);
+      wsum += w;
+      const float* po = p.part_o + prow(s0 + k) * D + lane * VPL;
+      if (VPL == 2) {
+        const float2 v = *reinterpret_cast<const float2*>(po);
+        acc[0] = fmaf(w, v.x, acc[0]);
+        acc[1] = fmaf(w, v.y, acc[1 % VPL]);
+      } else {
+        const float4 v = *reinterpret_cast<const float4*>(po);
+        acc[0] = fmaf(w, v.x, acc[0]);
+        acc[1 % VPL] = fmaf(w, v.y, acc[1 % VPL]);
+        acc[2 % VPL] = fmaf(w, v.z, acc[2 % VPL]);
+        acc[3 % VPL] = fmaf(w, v.w, acc[3 % VPL]);
+      }
+    }
   }
   const float inv = 1.f / wsum;
-  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + ((long long)row * p.heads + head) * D;
-#pragma unroll
-  for (int i = 0; i < D / 32; ++i) o[lane + 32 * i] = __float2bfloat16_rn(acc[i] * inv);
+  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + ((long long)row * p.heads + head) * D +
+                     lane * VPL;
+  if (VPL == 2) {
+    *reinterpret_cast<__nv_bfloat162*>(o) = __floats2bfloat162_rn(acc[0] * inv, acc[1] * inv);
+  } else {
+    *reinterpret_cast<__nv_bfloat162*>(o) = __floats2bfloat162_rn(acc[0] * inv, acc[1 % VPL] * inv);
+    *reinterpret_cast<__nv_bfloat162*>(o + 2) =
+        __floats2bfloat162_rn(acc[2 % VPL] * inv, acc[3 % VPL] * inv);
+  }
 }
 
 }  // namespace
@@ -825,31 +857,49 @@ cudaError_t prepare_attn_tc() {
 
 }  // namespace
 
+namespace {
+
+// Launch with programmatic stream serialisation: the kernel may be scheduled while the
+// previous kernel on the stream drains; it waits for it (griddepcontrol.wait) before
+// touching that kernel's results.
+template <typename K>
+cudaError_t launch_pdl(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       const AttnParams& p) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, p);
+}
+
+}  // namespace
+
 cudaError_t launch_attn_tc(const AttnParams& p, int head_dim, cudaStream_t s) {
   const dim3 grid(p.grid);
   cudaError_t e;
   if (head_dim == 64) {
     if ((e = prepare_attn_tc<64>()) != cudaSuccess) return e;
-    attn_tc_kernel<64><<<grid, kThreads, Cfg<64>::SMEM, s>>>(p);
-  } else if (head_dim == 128) {
-    if ((e = prepare_attn_tc<128>()) != cudaSuccess) return e;
-    attn_tc_kernel<128><<<grid, kThreads, Cfg<128>::SMEM, s>>>(p);
-  } else {
-    return cudaErrorInvalidValue;
+    return launch_pdl(attn_tc_kernel<64>, grid, dim3(kThreads), Cfg<64>::SMEM, s, p);
   }
-  return cudaGetLastError();
+  if (head_dim == 128) {
+    if ((e = prepare_attn_tc<128>()) != cudaSuccess) return e;
+    return launch_pdl(attn_tc_kernel<128>, grid, dim3(kThreads), Cfg<128>::SMEM, s, p);
+  }
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_attn_combine(const AttnParams& p, int head_dim, cudaStream_t s) {
   const long long warps = (long long)p.n_pairs * p.heads * (2 * BM);
-  const unsigned blocks = (unsigned)((warps * 32 + 255) / 256);
-  if (head_dim == 64)
-    attn_combine_kernel<64><<<blocks, 256, 0, s>>>(p);
-  else if (head_dim == 128)
-    attn_combine_kernel<128><<<blocks, 256, 0, s>>>(p);
-  else
-    return cudaErrorInvalidValue;
-  return cudaGetLastError();
+  const dim3 blocks((unsigned)((warps * 32 + 255) / 256));
+  if (head_dim == 64) return launch_pdl(attn_combine_kernel<64>, blocks, dim3(256), 0, s, p);
+  if (head_dim == 128) return launch_pdl(attn_combine_kernel<128>, blocks, dim3(256), 0, s, p);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace lbm

@@ -112,6 +112,10 @@ template <typename T, int CPR>
 __global__ void __launch_bounds__(kAppendThreads)
     rope_append_kernel(RopeTables rt, Pools pools, AppendArgs a) {
   constexpr int EPC = 16 / sizeof(T);
+  // launched as a programmatic dependent of the previous kernel on the stream (the previous
+  // frame's attention may still read the page and slots written here): wait for it to
+  // finish before touching memory; the launch itself already overlapped its tail
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const uint32_t per_tensor = (uint32_t)a.tokens * a.heads * CPR;
   const uint32_t total = 3u * per_tensor;
   const uint32_t stride_all = gridDim.x * blockDim.x * kAppendUnroll;
@@ -214,18 +218,25 @@ cudaError_t launch_rope_append(const RopeTables& rt, const Pools& pools, const A
   long long blocks = (chunks + per_block - 1) / per_block;
   if (blocks > 148 * 64) blocks = 148 * 64;
   if (blocks < 1) blocks = 1;
-  const dim3 grid((unsigned)blocks);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3((unsigned)blocks);
+  cfg.blockDim = dim3(kAppendThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (a.dtype == LBM_BF16 && cpr == 8)
-    rope_append_kernel<__nv_bfloat16, 8><<<grid, kAppendThreads, 0, s>>>(rt, pools, a);
-  else if (a.dtype == LBM_BF16 && cpr == 16)
-    rope_append_kernel<__nv_bfloat16, 16><<<grid, kAppendThreads, 0, s>>>(rt, pools, a);
-  else if (a.dtype == LBM_F32 && cpr == 16)
-    rope_append_kernel<float, 16><<<grid, kAppendThreads, 0, s>>>(rt, pools, a);
-  else if (a.dtype == LBM_F32 && cpr == 32)
-    rope_append_kernel<float, 32><<<grid, kAppendThreads, 0, s>>>(rt, pools, a);
-  else
-    return cudaErrorInvalidValue;
-  return cudaGetLastError();
+    return cudaLaunchKernelEx(&cfg, rope_append_kernel<__nv_bfloat16, 8>, rt, pools, a);
+  if (a.dtype == LBM_BF16 && cpr == 16)
+    return cudaLaunchKernelEx(&cfg, rope_append_kernel<__nv_bfloat16, 16>, rt, pools, a);
+  if (a.dtype == LBM_F32 && cpr == 16)
+    return cudaLaunchKernelEx(&cfg, rope_append_kernel<float, 16>, rt, pools, a);
+  if (a.dtype == LBM_F32 && cpr == 32)
+    return cudaLaunchKernelEx(&cfg, rope_append_kernel<float, 32>, rt, pools, a);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace lbm
