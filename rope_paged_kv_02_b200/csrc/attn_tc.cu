@@ -41,9 +41,6 @@ constexpr uint32_t kTmemCols = 512;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when max grows by > 2^8
 constexpr unsigned kFull = 0xffffffffu;
-// a waiting thread may sleep in mbarrier.try_wait up to this long before re-checking the
-// time limit, instead of spinning and taking issue slots from the softmax warps
-constexpr uint32_t kSuspendHintNs = 1000000;
 
 template <int D>
 struct Cfg {
@@ -84,14 +81,18 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
+// try_wait without a suspend-time hint: the thread may be suspended for a short,
+// system-defined time and resumes as soon as the phase completes.  (A long hint delayed the
+// wake-up by several hundred cycles after the completing arrival, on the critical path
+// between the softmax and MMA roles; spinning on test_wait took issue slots instead.)
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
+      : "r"(bar), "r"(parity)
       : "memory");
   return ok != 0;
 }
@@ -351,7 +352,7 @@ __device__ __forceinline__ int seg_nq(const AttnParams& p, const Segment& sg, in
   return min(2, q_tiles - 2 * seg_pair(p, sg));
 }
 
-// Persistent CTA c of p.grid walks the global work items [sk_lo(c), sk_lo(c+1)).  Every role
+// Persistent CTA c of p.grid walks the global work items [sk_start[c], sk_start[c+1]).  Every role
 // walks the same segments; barrier phases run on across segments (counters per role).
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -369,8 +370,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = __shfl_sync(0xffffffffu, (int)(threadIdx.x >> 5), 0);
   const int lane = threadIdx.x & 31;
   const int q_tiles = (p.tokens + BM - 1) / BM;
-  const int lo = (int)sk_lo(p.work, p.grid, blockIdx.x);
-  const int hi = (int)sk_lo(p.work, p.grid, blockIdx.x + 1);
+  const int lo = p.sk_start[blockIdx.x];
+  const int hi = p.sk_start[blockIdx.x + 1];
 
   const uint32_t sQ = smem_u32(smem + C::OFF_Q);
   const uint32_t sK = smem_u32(smem + C::OFF_K);
@@ -767,6 +768,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 // One warp per (unit, row of the pair).  Lane s loads the LSE of segment s (32 segments at a
 // time), the warp reduces max and weights with shuffles, then every lane loads its features
 // of all segments back to back, so the loads of a row overlap instead of chaining.
+// Largest c in [0, grid) with sk_start[c] <= x (binary search, warp-uniform).
+__device__ __forceinline__ int last_start_at_or_before(const AttnParams& p, int x) {
+  int lo = 0, hi = p.grid - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.sk_start[mid] <= x)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  return lo;
+}
+
 template <int D>
 __global__ void __launch_bounds__(256) attn_combine_kernel(const __grid_constant__ AttnParams p) {
   constexpr int VPL = D / 32;  // features per lane
@@ -783,13 +797,11 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const __grid_constant
   if (row >= p.tokens) return;
   const long long first = (long long)unit * p.n_tiles;
   const long long last = first + p.n_tiles - 1;
-  // CTAs whose share [sk_lo(c), sk_lo(c+1)) meets this unit: c0 .. c1
-  int c0 = (int)(first * p.grid / p.work);
-  while (c0 > 0 && sk_lo(p.work, p.grid, c0) > first) --c0;
-  while (sk_lo(p.work, p.grid, c0 + 1) <= first) ++c0;
-  int c1 = (int)(last * p.grid / p.work);
-  while (c1 + 1 < p.grid && sk_lo(p.work, p.grid, c1 + 1) <= last) ++c1;
-  while (c1 > c0 && sk_lo(p.work, p.grid, c1) > last) --c1;
+  // CTAs whose share [sk_start[c], sk_start[c+1]) meets this unit: c0 .. c1 (the shares are
+  // non-empty and increasing, so c0 and c1 are the last CTAs starting at or before the
+  // unit's first and last item)
+  const int c0 = last_start_at_or_before(p, (int)first);
+  const int c1 = last_start_at_or_before(p, (int)last);
   if (c1 == c0) return;  // one CTA did the whole unit and wrote the output itself
   const int nseg = c1 - c0 + 1;
   // partial row of segment (CTA c0 + s): slot unit + c

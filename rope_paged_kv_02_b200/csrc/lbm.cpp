@@ -137,7 +137,8 @@ int fill_attn_params(lbm_cache* c, const void* q, void* out, lbm::AttnParams& p)
   p.work = (long long)p.n_pairs * c->heads * p.n_tiles;
   if (p.work >= (1LL << 31)) return LBM_ERR_UNSUPPORTED;  // the kernel counts in 32 bits
   const long long want = c->forced_grid ? c->forced_grid : c->num_sms;
-  p.grid = (int)std::min<long long>(want, p.work);
+  p.grid = (int)std::min<long long>(std::min<long long>(want, p.work), lbm::kMaxGrid);
+  lbm::sk_partition(p);
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)c->head_dim));
   return LBM_OK;
 }
@@ -261,7 +262,7 @@ int lbm_cache_create(int heads, int head_dim, int patches_per_frame, int special
   cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device);
   if (const char* env = std::getenv("LBM_ATTN_GRID")) {
     const int v = std::atoi(env);
-    if (v >= 1 && v <= 4 * c->num_sms) c->forced_grid = v;
+    if (v >= 1 && v <= 4 * c->num_sms && v <= lbm::kMaxGrid) c->forced_grid = v;
   }
 
   const int P = scale_frames + sliding_window + 1;
@@ -379,7 +380,7 @@ int lbm_attend_frame(lbm_cache_t* c, const void* q, void* out, void* stream) {
     p.part_lse = c->part_lse;
     if (lbm::launch_attn_tc(p, c->head_dim, s) != cudaSuccess) return LBM_ERR_CUDA;
     ++c->launches;
-    if (lbm::sk_has_split(p.work, p.grid, p.n_tiles)) {
+    if (lbm::sk_has_split(p)) {
       if (lbm::launch_attn_combine(p, c->head_dim, s) != cudaSuccess) return LBM_ERR_CUDA;
       ++c->launches;
     }
@@ -424,7 +425,7 @@ int lbm_attend_frame_noalloc(lbm_cache_t* c, const void* q, void* out, void* str
   const int pst = fill_attn_params(c, q, out, p);
   if (pst != LBM_OK) return pst;
   const long long units = (long long)p.n_pairs * c->heads;
-  const bool split = lbm::sk_has_split(p.work, p.grid, p.n_tiles);
+  const bool split = lbm::sk_has_split(p);
   if (split && lbm::sk_scratch_floats(units, p.grid, c->head_dim) > scratch_floats)
     return LBM_ERR_CAPACITY;
   p.part_o = scratch;

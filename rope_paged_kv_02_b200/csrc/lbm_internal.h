@@ -43,17 +43,16 @@ struct AppendArgs {
 
 constexpr int kMaxPages = 1024;
 
+constexpr int kMaxGrid = 1024;  // persistent attention CTAs per launch, at most
+
 // Kernel parameter block of the paged attention (passed by value).
 // Stream-K partition of one frame's attention over `grid` persistent CTAs.  A unit is one
 // (pair of 128-row query tiles, head), unit u = head * n_pairs + pair; its key tiles are the
 // global work items [u * n_tiles, (u + 1) * n_tiles).  CTA c processes the contiguous items
-// [sk_lo(c), sk_lo(c + 1)), i.e. a run of segments (unit, key-tile range); a segment that
-// is a whole unit writes the final output, any other writes a partial (O, LSE) into slot
-// unit + c (dense: at most units + grid slots), merged by the combine kernel.
-__host__ __device__ inline long long sk_lo(long long work, int grid, int c) {
-  return (long long)c * work / grid;
-}
-
+// [sk_start[c], sk_start[c + 1]) (never empty), i.e. a run of segments (unit, key-tile
+// range); a segment that is a whole unit writes the final output, any other writes a
+// partial (O, LSE) into slot unit + c (dense: at most units + grid slots), merged by the
+// combine kernel.  The host places the boundaries by cost (sk_partition).
 struct AttnParams {
   CUtensorMap tm_q;      // q   {head_dim, heads, T}
   CUtensorMap tm_kp;     // K patch pool {head_dim, P*stride, heads}
@@ -77,6 +76,7 @@ struct AttnParams {
   int grid;              // persistent CTAs
   float scale_log2;      // log2(e) / sqrt(head_dim)
   uint16_t pages[kMaxPages];
+  int sk_start[kMaxGrid + 1];  // first work item of CTA c; sk_start[grid] = work
 };
 
 struct SimtParams {
@@ -108,10 +108,58 @@ cudaError_t launch_attn_combine(const AttnParams& p, int head_dim, cudaStream_t 
 inline size_t sk_scratch_floats(long long units, int grid, int head_dim) {
   return (size_t)(units + grid) * 256 * (size_t)(head_dim + 1);
 }
+// Relative costs of the stream-K partition, measured on the tensor-core kernel: a key-tile
+// step of a pair with two query tiles (both softmax warpgroups busy), a step of a pair with
+// a single query tile, and the pipeline refill at the start of every segment.
+constexpr long long kCostPairStep = 6;
+constexpr long long kCostSingleStep = 5;
+constexpr long long kCostSegment = 10;
+
+// Fills p.sk_start[0 .. p.grid] (needs p.n_tiles, n_pairs, heads, tokens, work, grid with
+// 1 <= grid <= min(work, kMaxGrid)): CTA c starts at the first item whose cost offset reaches
+// c / grid of the frame's total cost; then every CTA is given at least one item.
+inline void sk_partition(AttnParams& p) {
+  const int q_tiles = (p.tokens + 127) / 128;
+  const bool last_single = (q_tiles & 1) != 0;
+  const long long nt = p.n_tiles;
+  auto unit_cost = [&](int pair) {
+    const bool single = last_single && pair == p.n_pairs - 1;
+    return kCostSegment + nt * (single ? kCostSingleStep : kCostPairStep);
+  };
+  const long long per_head = (long long)(p.n_pairs - 1) * unit_cost(0) + unit_cost(p.n_pairs - 1);
+  const long long total = per_head * p.heads;
+  for (int c = 0; c <= p.grid; ++c) {
+    const long long v = (long long)((__int128)c * total / p.grid);
+    long long x;
+    if (c == p.grid) {
+      x = p.work;
+    } else {
+      const long long head = v / per_head;
+      long long r = v - head * per_head;
+      int pair = 0;
+      while (pair < p.n_pairs - 1 && r >= unit_cost(pair)) r -= unit_cost(pair++);
+      const long long w = last_single && pair == p.n_pairs - 1 ? kCostSingleStep : kCostPairStep;
+      // item t > 0 of the unit starts at cost kCostSegment + t * w (item 0 at 0)
+      long long t = r <= 0 ? 0 : (r - kCostSegment + w - 1) / w;
+      if (r > 0 && t < 1) t = 1;
+      if (t > nt) t = nt;
+      x = ((long long)head * p.n_pairs + pair) * nt + t;
+    }
+    p.sk_start[c] = (int)x;
+  }
+  // non-empty shares: strictly increasing starts, each leaving room for the CTAs after it
+  for (int c = 1; c < p.grid; ++c) {
+    long long x = p.sk_start[c];
+    if (x < (long long)p.sk_start[c - 1] + 1) x = p.sk_start[c - 1] + 1;
+    if (x > p.work - (p.grid - c)) x = p.work - (p.grid - c);
+    p.sk_start[c] = (int)x;
+  }
+}
+
 // true when some unit is shared by two CTAs (then the combine kernel must run)
-inline bool sk_has_split(long long work, int grid, int n_tiles) {
-  for (int c = 1; c < grid; ++c)
-    if (sk_lo(work, grid, c) % n_tiles != 0) return true;
+inline bool sk_has_split(const AttnParams& p) {
+  for (int c = 1; c < p.grid; ++c)
+    if (p.sk_start[c] % p.n_tiles != 0) return true;
   return false;
 }
 

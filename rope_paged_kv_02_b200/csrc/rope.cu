@@ -69,109 +69,100 @@ __device__ __forceinline__ uint32_t pack_bf(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&b);
 }
 
-// Rotates the 16-byte chunk starting at feature d0 of a token at (t, hh, ww).
+// Rotates the feature pairs of one 16-byte chunk by the given (cos, sin) per pair.
 template <typename T>
-__device__ __forceinline__ U4 rotate_chunk(const RopeTables& rt, U4 in, int d0, int t, int hh,
-                                           int ww);
+__device__ __forceinline__ U4 rotate_chunk(U4 in, const float2* cs);
 
 template <>
-__device__ __forceinline__ U4 rotate_chunk<__nv_bfloat16>(const RopeTables& rt, U4 in, int d0,
-                                                          int t, int hh, int ww) {
+__device__ __forceinline__ U4 rotate_chunk<__nv_bfloat16>(U4 in, const float2* cs) {
   // 8 bf16 = 4 pairs; pair u lives in word u (low half = x[2i], high half = x[2i+1]).
   uint32_t w[4] = {in.x, in.y, in.z, in.w};
-  const int i0 = d0 >> 1;
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
     float x0 = bf_lo(w[u]), x1 = bf_hi(w[u]);
-    rot(x0, x1, pair_cs(rt, i0 + u, t, hh, ww));
+    rot(x0, x1, cs[u]);
     w[u] = pack_bf(x0, x1);
   }
   return U4{w[0], w[1], w[2], w[3]};
 }
 
 template <>
-__device__ __forceinline__ U4 rotate_chunk<float>(const RopeTables& rt, U4 in, int d0, int t,
-                                                  int hh, int ww) {
+__device__ __forceinline__ U4 rotate_chunk<float>(U4 in, const float2* cs) {
   float x[4] = {__uint_as_float(in.x), __uint_as_float(in.y), __uint_as_float(in.z),
                 __uint_as_float(in.w)};
-  const int i0 = d0 >> 1;
-  rot(x[0], x[1], pair_cs(rt, i0, t, hh, ww));
-  rot(x[2], x[3], pair_cs(rt, i0 + 1, t, hh, ww));
+  rot(x[0], x[1], cs[0]);
+  rot(x[2], x[3], cs[1]);
   return U4{__float_as_uint(x[0]), __float_as_uint(x[1]), __float_as_uint(x[2]),
             __float_as_uint(x[3])};
 }
 
 constexpr int kAppendThreads = 256;
-constexpr int kAppendUnroll = 1;
 
-// One pass over the 3 * T * H * (D / EPC) 16-byte chunks of q, k, v (32-bit indices: a
-// frame is far below 2^31 chunks): tensor-major (q, k, v), then token, head, chunk, so
-// neighbouring threads touch neighbouring 16-byte chunks.  CPR = chunks per (token, head)
-// row is a compile-time power of two, so only the division by the head count is a real one.
-template <typename T, int CPR>
+// Thread (token j, 16-byte chunk c) of head group blockIdx.y handles HG consecutive heads:
+// the chunk's (cos, sin) pairs depend only on the token and the feature, so they and all the
+// index arithmetic are computed once and reused for q and k of every head of the group.
+// Lanes run over chunks first, then tokens, so a warp reads whole 128-byte rows of q, k, v
+// and, per head, writes consecutive rows of the frame's page.  All 3 * HG loads of a thread
+// are issued before the first rotation, to keep enough bytes in flight to cover HBM latency.
+template <typename T, int CPR, int HG>
 __global__ void __launch_bounds__(kAppendThreads)
     rope_append_kernel(RopeTables rt, Pools pools, AppendArgs a) {
-  constexpr int EPC = 16 / sizeof(T);
+  constexpr int EPC = 16 / sizeof(T);  // elements per 16-byte chunk
+  constexpr int NPC = EPC / 2;         // feature pairs per chunk
   // launched as a programmatic dependent of the previous kernel on the stream (the previous
   // frame's attention may still read the page and slots written here): wait for it to
   // finish before touching memory; the launch itself already overlapped its tail
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const uint32_t per_tensor = (uint32_t)a.tokens * a.heads * CPR;
-  const uint32_t total = 3u * per_tensor;
-  const uint32_t stride_all = gridDim.x * blockDim.x * kAppendUnroll;
-  for (uint32_t base = blockIdx.x * blockDim.x * kAppendUnroll + threadIdx.x; base < total;
-       base += stride_all) {
-    U4 val[kAppendUnroll];
-    // issue every load of this round before any arithmetic (memory-level parallelism)
+  const uint32_t items = (uint32_t)a.tokens * CPR;
+  const uint32_t idx = blockIdx.x * kAppendThreads + threadIdx.x;
+  if (idx >= items) return;
+  const int c = (int)(idx % CPR);
+  const int j = (int)(idx / CPR);
+  const int h0 = blockIdx.y * HG;
+
+  // sources: [tokens][heads][CPR] chunks
+  const size_t row_chunks = (size_t)a.heads * CPR;
+  const size_t src0 = (size_t)j * row_chunks + (size_t)h0 * CPR + c;
+  U4 vq[HG], vk[HG], vv[HG];
 #pragma unroll
-    for (int u = 0; u < kAppendUnroll; ++u) {
-      const uint32_t idx = base + u * blockDim.x;
-      if (idx < total) {
-        const uint32_t tensor = idx >= per_tensor ? (idx >= 2 * per_tensor ? 2u : 1u) : 0u;
-        const uint32_t rem = idx - tensor * per_tensor;
-        const char* src = tensor == 0 ? (const char*)a.q : tensor == 1 ? (const char*)a.k
-                                                                       : (const char*)a.v;
-        src += (size_t)rem * 16;
-        val[u] = tensor == 0 ? ld_plain(src) : ld_stream(src);
-      }
-    }
+  for (int u = 0; u < HG; ++u) {
+    vq[u] = ld_plain((const char*)a.q + (src0 + u * CPR) * 16);
+    vk[u] = ld_stream((const char*)a.k + (src0 + u * CPR) * 16);
+    vv[u] = ld_stream((const char*)a.v + (src0 + u * CPR) * 16);
+  }
+
+  int hh = 0, ww = 0;
+  const bool special = j < a.psi;
+  if (!special) {
+    const int pj = j - a.psi;
+    hh = 1 + pj / rt.ppw;
+    ww = 1 + pj - (hh - 1) * rt.ppw;
+  }
+  float2 cs[NPC];
+  const int i0 = c * NPC;
 #pragma unroll
-    for (int u = 0; u < kAppendUnroll; ++u) {
-      const uint32_t idx = base + u * blockDim.x;
-      if (idx >= total) continue;
-      const uint32_t tensor = idx >= per_tensor ? (idx >= 2 * per_tensor ? 2u : 1u) : 0u;
-      const uint32_t rem = idx - tensor * per_tensor;
-      const int c = (int)(rem % CPR);
-      const uint32_t th = rem / CPR;
-      const int j = (int)(th / (uint32_t)a.heads);
-      const int h = (int)(th - (uint32_t)j * a.heads);
-      const int d0 = c * EPC;
-      U4 out = val[u];
-      if (tensor < 2) {
-        int hh = 0, ww = 0;
-        if (j >= a.psi) {
-          const int pj = j - a.psi;
-          hh = 1 + pj / rt.ppw;
-          ww = 1 + pj - (hh - 1) * rt.ppw;
-        }
-        out = rotate_chunk<T>(rt, out, d0, a.frame, hh, ww);
-      }
-      char* dst;
-      if (tensor == 0) {
-        dst = (char*)a.q + (size_t)rem * 16;
-      } else {
-        const bool special = j < a.psi;
-        void* pool = special ? (tensor == 1 ? pools.k_special : pools.v_special)
-                             : (tensor == 1 ? pools.k_patch : pools.v_patch);
-        size_t row;
-        if (special)
-          row = (size_t)h * pools.spec_cap + a.special_slot + j;
-        else
-          row = ((size_t)h * pools.num_pages + a.page) * pools.page_stride + (j - a.psi);
-        dst = (char*)pool + (row * CPR + c) * 16;
-      }
-      st_plain(dst, out);
-    }
+  for (int u = 0; u < NPC; ++u) cs[u] = pair_cs(rt, i0 + u, a.frame, hh, ww);
+
+  // destinations: the special stream [heads][spec_cap] or the frame's page
+  // [heads][num_pages * page_stride] rows of CPR chunks
+  size_t dst0, head_step;
+  char *kpool, *vpool;
+  if (special) {
+    kpool = (char*)pools.k_special;
+    vpool = (char*)pools.v_special;
+    head_step = (size_t)pools.spec_cap * CPR;
+    dst0 = ((size_t)h0 * pools.spec_cap + a.special_slot + j) * CPR + c;
+  } else {
+    kpool = (char*)pools.k_patch;
+    vpool = (char*)pools.v_patch;
+    head_step = (size_t)pools.num_pages * pools.page_stride * CPR;
+    dst0 = (((size_t)h0 * pools.num_pages + a.page) * pools.page_stride + (j - a.psi)) * CPR + c;
+  }
+#pragma unroll
+  for (int u = 0; u < HG; ++u) {
+    st_plain((char*)a.q + (src0 + u * CPR) * 16, rotate_chunk<T>(vq[u], cs));
+    st_plain(kpool + (dst0 + u * head_step) * 16, rotate_chunk<T>(vk[u], cs));
+    st_plain(vpool + (dst0 + u * head_step) * 16, vv[u]);
   }
 }
 
@@ -212,30 +203,35 @@ cudaError_t launch_rope_append(const RopeTables& rt, const Pools& pools, const A
                                cudaStream_t s) {
   const int esz = a.dtype == LBM_BF16 ? 2 : 4;
   const int cpr = a.head_dim * esz / 16;
-  const long long chunks = 3LL * a.tokens * a.heads * cpr;
-  if (chunks >= (1LL << 31)) return cudaErrorInvalidValue;
-  const long long per_block = (long long)kAppendThreads * kAppendUnroll;
-  long long blocks = (chunks + per_block - 1) / per_block;
-  if (blocks > 148 * 64) blocks = 148 * 64;
-  if (blocks < 1) blocks = 1;
+  const long long items = (long long)a.tokens * cpr;
+  if (items <= 0 || 3LL * items * a.heads >= (1LL << 31)) return cudaErrorInvalidValue;
+  // heads per thread: 4 when that still leaves at least ~one block of 128 threads per SM,
+  // else fewer (small frames need the threads more than the reuse)
+  int hg = 1;
+  if (a.heads % 4 == 0 && items * (a.heads / 4) >= 148LL * 128)
+    hg = 4;
+  else if (a.heads % 2 == 0 && items * (a.heads / 2) >= 148LL * 128)
+    hg = 2;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.gridDim = dim3((unsigned)blocks);
+  cfg.gridDim = dim3((unsigned)((items + kAppendThreads - 1) / kAppendThreads),
+                     (unsigned)(a.heads / hg));
   cfg.blockDim = dim3(kAppendThreads);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (a.dtype == LBM_BF16 && cpr == 8)
-    return cudaLaunchKernelEx(&cfg, rope_append_kernel<__nv_bfloat16, 8>, rt, pools, a);
-  if (a.dtype == LBM_BF16 && cpr == 16)
-    return cudaLaunchKernelEx(&cfg, rope_append_kernel<__nv_bfloat16, 16>, rt, pools, a);
-  if (a.dtype == LBM_F32 && cpr == 16)
-    return cudaLaunchKernelEx(&cfg, rope_append_kernel<float, 16>, rt, pools, a);
-  if (a.dtype == LBM_F32 && cpr == 32)
-    return cudaLaunchKernelEx(&cfg, rope_append_kernel<float, 32>, rt, pools, a);
+#define LBM_APPEND_LAUNCH(T, C)                                                           \
+  if (hg == 4) return cudaLaunchKernelEx(&cfg, rope_append_kernel<T, C, 4>, rt, pools, a); \
+  if (hg == 2) return cudaLaunchKernelEx(&cfg, rope_append_kernel<T, C, 2>, rt, pools, a); \
+  return cudaLaunchKernelEx(&cfg, rope_append_kernel<T, C, 1>, rt, pools, a);
+  if (a.dtype == LBM_BF16 && cpr == 8) { LBM_APPEND_LAUNCH(__nv_bfloat16, 8) }
+  if (a.dtype == LBM_BF16 && cpr == 16) { LBM_APPEND_LAUNCH(__nv_bfloat16, 16) }
+  if (a.dtype == LBM_F32 && cpr == 16) { LBM_APPEND_LAUNCH(float, 16) }
+  if (a.dtype == LBM_F32 && cpr == 32) { LBM_APPEND_LAUNCH(float, 32) }
+#undef LBM_APPEND_LAUNCH
   return cudaErrorInvalidValue;
 }
 
