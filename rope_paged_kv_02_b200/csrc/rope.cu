@@ -205,12 +205,13 @@ cudaError_t launch_rope_append(const RopeTables& rt, const Pools& pools, const A
   const int cpr = a.head_dim * esz / 16;
   const long long items = (long long)a.tokens * cpr;
   if (items <= 0 || 3LL * items * a.heads >= (1LL << 31)) return cudaErrorInvalidValue;
-  // heads per thread: 4 when that still leaves at least ~one block of 128 threads per SM,
-  // else fewer (small frames need the threads more than the reuse)
+  // heads per thread: the most (4, 2, 1) that still leaves two blocks of 256 threads per SM
+  // in flight (small frames need the threads to cover HBM latency more than the reuse)
+  const long long min_threads = 148LL * 2 * kAppendThreads;
   int hg = 1;
-  if (a.heads % 4 == 0 && items * (a.heads / 4) >= 148LL * 128)
+  if (a.heads % 4 == 0 && items * (a.heads / 4) >= min_threads)
     hg = 4;
-  else if (a.heads % 2 == 0 && items * (a.heads / 2) >= 148LL * 128)
+  else if (a.heads % 2 == 0 && items * (a.heads / 2) >= min_threads)
     hg = 2;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
