@@ -763,11 +763,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Merges the partial results of the units that span more than one CTA:
-// out[row][h] = sum_s w_s o_s / sum_s w_s with w_s = 2^(lse_s - max_s lse_s).
-// One warp per (unit, row of the pair).  Lane s loads the LSE of segment s (32 segments at a
-// time), the warp reduces max and weights with shuffles, then every lane loads its features
-// of all segments back to back, so the loads of a row overlap instead of chaining.
 // Largest c in [0, grid) with sk_start[c] <= x (binary search, warp-uniform).
 __device__ __forceinline__ int last_start_at_or_before(const AttnParams& p, int x) {
   int lo = 0, hi = p.grid - 1;
@@ -781,73 +776,92 @@ __device__ __forceinline__ int last_start_at_or_before(const AttnParams& p, int 
   return lo;
 }
 
+// Merges the partial results of the units that span more than one CTA:
+// out[row][h] = sum_s w_s o_s / sum_s w_s with w_s = 2^(lse_s - max_s lse_s).
+// One warp per (unit, two rows of the pair): each half-warp owns one row, its 16 lanes hold
+// D / 16 features each.  Lane s of a half loads the LSE of segment s (16 at a time), the half
+// reduces max and weights with shuffles, then the O rows of four segments are loaded before
+// any is used, so a row costs about two L2 round trips.
 template <int D>
 __global__ void __launch_bounds__(256) attn_combine_kernel(const __grid_constant__ AttnParams p) {
-  constexpr int VPL = D / 32;  // features per lane
-  asm volatile("griddepcontrol.wait;" ::: "memory");  // partials of the attention kernel
+  constexpr int VPL = D / 16;  // features per lane
+  constexpr int V4 = VPL / 4;  // float4 loads per lane and segment
   const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
+  const int half = lane >> 4;
+  const int hl = lane & 15;
   const long long units = (long long)p.n_pairs * p.heads;
-  if (gw >= units * (2 * BM)) return;
-  const int unit = (int)(gw / (2 * BM));
-  const int row_in_pair = (int)(gw - (long long)unit * (2 * BM));
+  if (gw >= units * BM) return;  // BM warps x 2 rows = the 256 rows of a unit
+  const int unit = (int)(gw / BM);
+  const int row_in_pair = (int)(gw - (long long)unit * BM) * 2 + half;
   const int pair = unit % p.n_pairs;
   const int head = unit / p.n_pairs;
   const int row = 2 * pair * BM + row_in_pair;
-  if (row >= p.tokens) return;
-  const long long first = (long long)unit * p.n_tiles;
-  const long long last = first + p.n_tiles - 1;
+  const int first = unit * p.n_tiles;
   // CTAs whose share [sk_start[c], sk_start[c+1]) meets this unit: c0 .. c1 (the shares are
   // non-empty and increasing, so c0 and c1 are the last CTAs starting at or before the
   // unit's first and last item)
-  const int c0 = last_start_at_or_before(p, (int)first);
-  const int c1 = last_start_at_or_before(p, (int)last);
+  const int c0 = last_start_at_or_before(p, first);
+  const int c1 = last_start_at_or_before(p, first + p.n_tiles - 1);
   if (c1 == c0) return;  // one CTA did the whole unit and wrote the output itself
+  // the index arithmetic above reads only kernel parameters and overlapped the attention
+  // kernel's tail; its partials are read only after it has completed
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const bool valid = row < p.tokens;  // rows past the frame have no partials
   const int nseg = c1 - c0 + 1;
   // partial row of segment (CTA c0 + s): slot unit + c
   auto prow = [&](int s) { return ((long long)unit + c0 + s) * (2 * BM) + row_in_pair; };
   float mx = -INFINITY;
-  for (int s0 = 0; s0 < nseg; s0 += 32) {
-    const float v = s0 + lane < nseg ? p.part_lse[prow(s0 + lane)] : -INFINITY;
+  for (int s0 = 0; s0 < nseg; s0 += 16) {
+    const float v = valid && s0 + hl < nseg ? p.part_lse[prow(s0 + hl)] : -INFINITY;
     mx = fmaxf(mx, v);
   }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  for (int o = 8; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   float acc[VPL];
 #pragma unroll
   for (int i = 0; i < VPL; ++i) acc[i] = 0.f;
   float wsum = 0.f;
-  for (int s0 = 0; s0 < nseg; s0 += 32) {
+  for (int s0 = 0; s0 < nseg; s0 += 16) {
     const float w_lane =
-        s0 + lane < nseg ? exp2f(p.part_lse[prow(s0 + lane)] - mx) : 0.f;
-    const int cnt = min(32, nseg - s0);
-    for (int k = 0; k < cnt; ++k) {
-      const float w = __shfl_sync(0xffffffffu, w_lane, k);
-      wsum += w;
-      const float* po = p.part_o + prow(s0 + k) * D + lane * VPL;
-      if (VPL == 2) {
-        const float2 v = *reinterpret_cast<const float2*>(po);
-        acc[0] = fmaf(w, v.x, acc[0]);
-        acc[1] = fmaf(w, v.y, acc[1 % VPL]);
-      } else {
-        const float4 v = *reinterpret_cast<const float4*>(po);
-        acc[0] = fmaf(w, v.x, acc[0]);
-        acc[1 % VPL] = fmaf(w, v.y, acc[1 % VPL]);
-        acc[2 % VPL] = fmaf(w, v.z, acc[2 % VPL]);
-        acc[3 % VPL] = fmaf(w, v.w, acc[3 % VPL]);
+        valid && s0 + hl < nseg ? exp2f(p.part_lse[prow(s0 + hl)] - mx) : 0.f;
+    const int cnt = min(16, nseg - s0);  // the same for both halves (one unit per warp)
+    for (int k0 = 0; k0 < cnt; k0 += 4) {
+      float4 v[4][V4];
+      float w[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int k = k0 + u;
+        w[u] = __shfl_sync(0xffffffffu, w_lane, (half << 4) + min(k, cnt - 1));
+        const float4* po = reinterpret_cast<const float4*>(
+            p.part_o + prow(s0 + min(k, cnt - 1)) * D + hl * VPL);
+#pragma unroll
+        for (int q = 0; q < V4; ++q)
+          v[u][q] = valid && k < cnt ? po[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (k0 + u >= cnt) break;
+        wsum += w[u];
+#pragma unroll
+        for (int q = 0; q < V4; ++q) {
+          acc[4 * q] = fmaf(w[u], v[u][q].x, acc[4 * q]);
+          acc[4 * q + 1] = fmaf(w[u], v[u][q].y, acc[4 * q + 1]);
+          acc[4 * q + 2] = fmaf(w[u], v[u][q].z, acc[4 * q + 2]);
+          acc[4 * q + 3] = fmaf(w[u], v[u][q].w, acc[4 * q + 3]);
+        }
       }
     }
   }
+  if (!valid) return;
   const float inv = 1.f / wsum;
   __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + ((long long)row * p.heads + head) * D +
-                     lane * VPL;
-  if (VPL == 2) {
-    *reinterpret_cast<__nv_bfloat162*>(o) = __floats2bfloat162_rn(acc[0] * inv, acc[1] * inv);
-  } else {
-    *reinterpret_cast<__nv_bfloat162*>(o) = __floats2bfloat162_rn(acc[0] * inv, acc[1 % VPL] * inv);
-    *reinterpret_cast<__nv_bfloat162*>(o + 2) =
-        __floats2bfloat162_rn(acc[2 % VPL] * inv, acc[3 % VPL] * inv);
-  }
+                     hl * VPL;
+#pragma unroll
+  for (int q = 0; q < V4; ++q)
+    *reinterpret_cast<uint2*>(o + 4 * q) =
+        make_uint2(pack_bf16(acc[4 * q] * inv, acc[4 * q + 1] * inv),
+                   pack_bf16(acc[4 * q + 2] * inv, acc[4 * q + 3] * inv));
 }
 
 }  // namespace
@@ -907,7 +921,7 @@ cudaError_t launch_attn_tc(const AttnParams& p, int head_dim, cudaStream_t s) {
 }
 
 cudaError_t launch_attn_combine(const AttnParams& p, int head_dim, cudaStream_t s) {
-  const long long warps = (long long)p.n_pairs * p.heads * (2 * BM);
+  const long long warps = (long long)p.n_pairs * p.heads * BM;  // two rows per warp
   const dim3 blocks((unsigned)((warps * 32 + 255) / 256));
   if (head_dim == 64) return launch_pdl(attn_combine_kernel<64>, blocks, dim3(256), 0, s, p);
   if (head_dim == 128) return launch_pdl(attn_combine_kernel<128>, blocks, dim3(256), 0, s, p);
