@@ -124,10 +124,14 @@ LBM_API int lbm_cache_create(int heads, int head_dim, int patches_per_frame, int
  *          frame's patch page (tokens >= 6) and the next 6 slots of the special stream
  *   frame_idx    strictly greater than the previous frame's, and < rope's ppf
  *   is_keyframe  1: the frame is kept after its attention; 0: rolled back after it
- *                ([KVBenefits] "Reduced KV Growth via Keyframe Streaming")
+ *                ([KVBenefits] "Reduced KV Growth via Keyframe Streaming");
+ *                LBM_KEYFRAME_DEFERRED: decided after the attention by lbm_commit_frame
+ *                ([KVBenefits] "Dynamic Keyframe Selection": selection by what the frame
+ *                shows); other values: LBM_ERR_INVALID
  * One kernel launch.  Errors: LBM_ERR_SEQUENCE if a frame is already pending or frame_idx
  * does not increase or is >= ppf; LBM_ERR_CAPACITY for a keyframe when max_frames keyframes
  * are committed. */
+#define LBM_KEYFRAME_DEFERRED 2
 LBM_API int lbm_append_frame(lbm_cache_t* cache, void* q, const void* k, const void* v,
                      long long frame_idx, int is_keyframe, void* stream);
 
@@ -135,12 +139,22 @@ LBM_API int lbm_append_frame(lbm_cache_t* cache, void* q, const void* k, const v
  * scale pages -> window pages (oldest first) -> the frame's own page -> all special tokens
  * ([3DRoPE-KV] "Attention Computation with Cached RoPE"); a frame's own tokens all see each
  * other; softmax scale 1/sqrt(head_dim).  Then commits the frame (keyframe; deferred
- * eviction) or rolls it back ([KVBenefits] "Dynamic Keyframe Selection").
+ * eviction) or rolls it back ([KVBenefits] "Dynamic Keyframe Selection"); a frame appended
+ * with LBM_KEYFRAME_DEFERRED stays pending until lbm_commit_frame.
  *   q    device [T][heads][head_dim], the q rotated by lbm_append_frame
  *   out  device [T][heads][head_dim], written
  * bf16: one tcgen05 kernel launch, plus one combine launch when the keys are split across
- * CTAs.  Errors: LBM_ERR_SEQUENCE if no frame is pending. */
+ * CTAs.  Errors: LBM_ERR_SEQUENCE if no frame is pending or the pending frame has already
+ * been attended. */
 LBM_API int lbm_attend_frame(lbm_cache_t* cache, const void* q, void* out, void* stream);
+
+/* Keep (keep != 0) or drop the pending frame appended with LBM_KEYFRAME_DEFERRED, after its
+ * attention ([KVBenefits] "Dynamic Keyframe Selection": a kept frame triggers the deferred
+ * eviction, a dropped frame's tentative entry is rolled back).  The resulting page table is
+ * the one an up-front is_keyframe = keep would have given.  Host-only; no GPU work.
+ * Errors: LBM_ERR_SEQUENCE unless such a frame is pending and attended; LBM_ERR_CAPACITY
+ * when keep and max_frames keyframes are committed (the frame stays pending: drop it). */
+LBM_API int lbm_commit_frame(lbm_cache_t* cache, int keep);
 
 /* Like lbm_attend_frame, for callers that may not allocate device memory while frames
  * stream (a runtime that owns the whole GPU through its own pool and budget, or a real-time
@@ -227,9 +241,12 @@ LBM_API int lbm_pager_append(lbm_pager_t* pager, long long frame_idx, int is_key
  * pages[0..capacity), their count, and the visible special tokens (committed + own). */
 LBM_API int lbm_pager_visible(const lbm_pager_t* pager, int* pages, int capacity, int* n_pages,
                       int* n_special, int* last_page_len);
-/* Commit (keyframe) or roll back (non-keyframe) the pending frame; *evicted receives the
- * page returned to the free list by deferred eviction, or -1. */
+/* The pending frame's attention is done: commit (keyframe) or roll back (non-keyframe) it;
+ * *evicted receives the page returned to the free list by deferred eviction, or -1.  A frame
+ * appended with LBM_KEYFRAME_DEFERRED only becomes attended (*evicted = -1). */
 LBM_API int lbm_pager_finish(lbm_pager_t* pager, int* evicted);
+/* Keep or drop an attended LBM_KEYFRAME_DEFERRED frame, as lbm_commit_frame. */
+LBM_API int lbm_pager_commit(lbm_pager_t* pager, int keep, int* evicted);
 LBM_API int lbm_pager_reset(lbm_pager_t* pager);
 LBM_API int lbm_pager_state(const lbm_pager_t* pager, lbm_cache_state_t* state);
 LBM_API void lbm_pager_destroy(lbm_pager_t* pager);

@@ -27,6 +27,11 @@ Readings (listed in DESIGN.md):
   P = scale_frames + sliding_window + 1.  Evicted and rolled-back pages are pushed on top.
 * The special stream is paged in pages of ``SPECIAL_PAGE`` = 128 tokens; the visible
   special tokens are the committed ones plus the current frame's.
+* The keep / drop decision may also be taken after the frame's attention ([KVBenefits]
+  "Dynamic Keyframe Selection" decides from what the frame shows): the frame is appended
+  undecided (``is_keyframe=None``) and ``finish(keep)`` commits or rolls it back.  Keeping
+  it then needs room in the special stream; otherwise the frame stays pending.  The result
+  is the state an up-front decision ``is_keyframe=keep`` would have given.
 """
 
 from __future__ import annotations
@@ -95,9 +100,10 @@ class PagedRetention:
         self.pending = None
         self.last_frame = -1
 
-    def append(self, frame_idx: int, is_keyframe: bool) -> tuple[int, int]:
+    def append(self, frame_idx: int, is_keyframe: bool | None) -> tuple[int, int]:
         """Tentatively place frame_idx: pop a patch page, reserve 6 special slots.
 
+        ``is_keyframe=None`` leaves the keep / drop decision to ``finish(keep)``.
         Returns (patch page id, first special slot).
         """
         if self.pending is not None:
@@ -107,7 +113,7 @@ class PagedRetention:
         if is_keyframe and len(self.committed) >= self.max_frames:
             raise CapacityError("special stream full")
         page = self.free.pop()
-        self.pending = (page, int(frame_idx), bool(is_keyframe))
+        self.pending = (page, int(frame_idx), None if is_keyframe is None else bool(is_keyframe))
         self.last_frame = int(frame_idx)
         return page, self.n_special
 
@@ -126,16 +132,23 @@ class PagedRetention:
             last_page_len=n_sp - SPECIAL_PAGE * (pages - 1),
         )
 
-    def finish(self) -> int | None:
+    def finish(self, keep: bool | None = None) -> int | None:
         """After the pending frame's attention: commit a keyframe or roll back.
 
         Commit fills scale first, then the window; a window longer than sliding_window
         returns its oldest page to the free stack (deferred eviction).  Returns the evicted
-        page, or None.  Roll-back returns the frame's page and drops its specials.
+        page, or None.  Roll-back returns the frame's page and drops its specials.  A frame
+        appended undecided needs ``keep``; one decided at append must not get it.
         """
         if self.pending is None:
             raise SequenceError("finish without append")
         page, frame, key = self.pending
+        if (key is None) == (keep is None):
+            raise SequenceError("decide a frame exactly once: at append or at finish")
+        if key is None:
+            if keep and len(self.committed) >= self.max_frames:
+                raise CapacityError("special stream full")
+            key = bool(keep)
         self.pending = None
         evicted = None
         if key:

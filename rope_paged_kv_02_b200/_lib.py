@@ -34,12 +34,22 @@ LBM_MAX_PAGES = 1024
 SYMBOLS = [
     "lbm_rope3d_tables", "lbm_rope3d_expand", "lbm_rope_destroy",
     "lbm_cache_create", "lbm_append_frame", "lbm_attend_frame", "lbm_attend_frame_noalloc",
-    "lbm_cache_reset",
+    "lbm_commit_frame", "lbm_cache_reset",
     "lbm_cache_state", "lbm_cache_read_kv", "lbm_cache_check", "lbm_cache_destroy",
     "lbm_status_string",
     "lbm_pager_create", "lbm_pager_append", "lbm_pager_visible", "lbm_pager_finish",
-    "lbm_pager_reset", "lbm_pager_state", "lbm_pager_destroy",
+    "lbm_pager_commit", "lbm_pager_reset", "lbm_pager_state", "lbm_pager_destroy",
 ]
+
+
+LBM_KEYFRAME_DEFERRED = 2
+
+
+def _keyframe_mode(is_keyframe) -> int:
+    """True -> 1, False -> 0, None -> LBM_KEYFRAME_DEFERRED (decided after attention)."""
+    if is_keyframe is None:
+        return LBM_KEYFRAME_DEFERRED
+    return 1 if is_keyframe else 0
 
 
 class LbmError(RuntimeError):
@@ -87,6 +97,7 @@ def load() -> ctypes.CDLL:
     lib.lbm_append_frame.argtypes = [c_void, c_void, c_void, c_void, c_ll, c_int, c_void]
     lib.lbm_attend_frame.argtypes = [c_void, c_void, c_void, c_void]
     lib.lbm_attend_frame_noalloc.argtypes = [c_void, c_void, c_void, c_void]
+    lib.lbm_commit_frame.argtypes = [c_void, c_int]
     lib.lbm_cache_reset.argtypes = [c_void]
     lib.lbm_cache_state.argtypes = [c_void, ctypes.POINTER(CacheState)]
     lib.lbm_cache_read_kv.argtypes = [c_void, c_int, c_int, c_int, c_void]
@@ -99,6 +110,7 @@ def load() -> ctypes.CDLL:
     lib.lbm_pager_append.argtypes = [c_void, c_ll, c_int, pint, pint]
     lib.lbm_pager_visible.argtypes = [c_void, pint, c_int, pint, pint, pint]
     lib.lbm_pager_finish.argtypes = [c_void, pint]
+    lib.lbm_pager_commit.argtypes = [c_void, c_int, pint]
     lib.lbm_pager_reset.argtypes = [c_void]
     lib.lbm_pager_state.argtypes = [c_void, ctypes.POINTER(CacheState)]
     lib.lbm_pager_destroy.argtypes = [c_void]
@@ -153,7 +165,9 @@ def _state_dict(fill, capacity: int) -> dict:
         "free": list(fp[:st.n_free]),
         "n_special": st.n_special, "special_pages": st.special_pages,
         "last_page_len": st.last_page_len, "pending": bool(st.pending),
-        "pending_page": st.pending_page, "pending_is_keyframe": bool(st.pending_is_keyframe),
+        "pending_page": st.pending_page,
+        "pending_is_keyframe": (None if st.pending_is_keyframe == LBM_KEYFRAME_DEFERRED
+                                else bool(st.pending_is_keyframe)),
         "pending_frame": st.pending_frame, "last_frame": st.last_frame,
         "device_bytes": st.device_bytes, "kernel_launches": st.kernel_launches,
     }
@@ -211,10 +225,14 @@ class PagedKVCache:
     def tokens(self) -> int:
         return self.psi + self.patches
 
-    def append_frame(self, q, k, v, frame_idx: int, is_keyframe: bool, stream=None) -> None:
+    def append_frame(self, q, k, v, frame_idx: int, is_keyframe, stream=None) -> None:
+        """is_keyframe: True / False, or None to decide after attention (commit_frame)."""
         _check(load().lbm_append_frame(self.handle, _ptr(q), _ptr(k), _ptr(v), int(frame_idx),
-                                       1 if is_keyframe else 0, _stream(stream)),
+                                       _keyframe_mode(is_keyframe), _stream(stream)),
                "lbm_append_frame")
+
+    def commit_frame(self, keep: bool) -> None:
+        _check(load().lbm_commit_frame(self.handle, 1 if keep else 0), "lbm_commit_frame")
 
     def attend_frame(self, q, out, stream=None) -> None:
         _check(load().lbm_attend_frame(self.handle, _ptr(q), _ptr(out), _stream(stream)),
@@ -262,12 +280,18 @@ class Pager:
         self.handle = h
         self.num_pages = scale_frames + sliding_window + 1
 
-    def append(self, frame_idx: int, is_keyframe: bool) -> tuple[int, int]:
+    def append(self, frame_idx: int, is_keyframe) -> tuple[int, int]:
         page, slot = ctypes.c_int(), ctypes.c_int()
-        _check(load().lbm_pager_append(self.handle, int(frame_idx), 1 if is_keyframe else 0,
+        _check(load().lbm_pager_append(self.handle, int(frame_idx), _keyframe_mode(is_keyframe),
                                        ctypes.byref(page), ctypes.byref(slot)),
                "lbm_pager_append")
         return page.value, slot.value
+
+    def commit(self, keep: bool) -> int:
+        ev = ctypes.c_int()
+        _check(load().lbm_pager_commit(self.handle, 1 if keep else 0, ctypes.byref(ev)),
+               "lbm_pager_commit")
+        return ev.value
 
     def visible(self) -> tuple[list, int, int]:
         cap = self.num_pages

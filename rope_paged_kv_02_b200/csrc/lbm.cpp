@@ -330,9 +330,10 @@ int lbm_append_frame(lbm_cache_t* c, void* q, const void* k, const void* v, long
                      int is_keyframe, void* stream) {
   if (!c || !q || !k || !v || !aligned16(q) || !aligned16(k) || !aligned16(v))
     return LBM_ERR_INVALID;
+  if (is_keyframe < 0 || is_keyframe > LBM_KEYFRAME_DEFERRED) return LBM_ERR_INVALID;
   if (frame_idx < 0 || frame_idx >= c->rope->t.ppf) return LBM_ERR_SEQUENCE;
   int page = -1, slot = -1;
-  switch (c->pager.peek_append(frame_idx, is_keyframe != 0, &page, &slot)) {
+  switch (c->pager.peek_append(frame_idx, is_keyframe, &page, &slot)) {
     case lbm::PagerStatus::kOk: break;
     case lbm::PagerStatus::kSequence: return LBM_ERR_SEQUENCE;
     case lbm::PagerStatus::kCapacity: return LBM_ERR_CAPACITY;
@@ -355,15 +356,27 @@ int lbm_append_frame(lbm_cache_t* c, void* q, const void* k, const void* v, long
   if (lbm::launch_rope_append(c->rope->t, c->pools, a, s) != cudaSuccess) return LBM_ERR_CUDA;
   ++c->launches;
   order_after(c, s);
-  c->pager.append(frame_idx, is_keyframe != 0, &page, &slot);
+  c->pager.append(frame_idx, is_keyframe, &page, &slot);
   return LBM_OK;
+}
+
+int lbm_commit_frame(lbm_cache_t* c, int keep) {
+  if (!c) return LBM_ERR_INVALID;
+  int evicted = -1;
+  switch (c->pager.commit(keep != 0, &evicted)) {
+    case lbm::PagerStatus::kOk: return LBM_OK;
+    case lbm::PagerStatus::kSequence: return LBM_ERR_SEQUENCE;
+    case lbm::PagerStatus::kCapacity: return LBM_ERR_CAPACITY;
+  }
+  return LBM_ERR_INVALID;
 }
 
 int lbm_attend_frame(lbm_cache_t* c, const void* q, void* out, void* stream) {
   if (!c || !q || !out || !aligned16(q) || !aligned16(out)) return LBM_ERR_INVALID;
   std::vector<int> pages;
   int n_sp = 0, last_len = 0;
-  if (c->pager.visible(&pages, &n_sp, &last_len) != lbm::PagerStatus::kOk)
+  if (!c->pager.awaiting_attention() ||
+      c->pager.visible(&pages, &n_sp, &last_len) != lbm::PagerStatus::kOk)
     return LBM_ERR_SEQUENCE;
   if (use_device(c->device) != LBM_OK) return LBM_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -415,7 +428,7 @@ int lbm_attend_frame(lbm_cache_t* c, const void* q, void* out, void* stream) {
 int lbm_attend_frame_noalloc(lbm_cache_t* c, const void* q, void* out, void* stream) {
   if (!c || !q || !out || !aligned16(q) || !aligned16(out)) return LBM_ERR_INVALID;
   if (c->dtype != LBM_BF16) return LBM_ERR_UNSUPPORTED;
-  if (!c->pager.pending()) return LBM_ERR_SEQUENCE;
+  if (!c->pager.awaiting_attention()) return LBM_ERR_SEQUENCE;
   if (use_device(c->device) != LBM_OK) return LBM_ERR_CUDA;
   float* scratch = nullptr;
   size_t scratch_floats = 0;

@@ -27,28 +27,32 @@ void Pager::reset() {
   pending_ = false;
   pending_page_ = -1;
   pending_key_ = false;
+  deferred_ = false;
+  attended_ = false;
   pending_frame_ = -1;
   last_frame_ = -1;
 }
 
-PagerStatus Pager::peek_append(long long frame_idx, bool is_keyframe, int* page,
+PagerStatus Pager::peek_append(long long frame_idx, int mode, int* page,
                                int* special_slot) const {
   if (pending_ || frame_idx <= last_frame_) return PagerStatus::kSequence;
-  if (is_keyframe && committed_ >= max_frames_) return PagerStatus::kCapacity;
+  if (mode == 1 && committed_ >= max_frames_) return PagerStatus::kCapacity;
   *page = free_.back();
   *special_slot = n_special_;
   return PagerStatus::kOk;
 }
 
-PagerStatus Pager::append(long long frame_idx, bool is_keyframe, int* page, int* special_slot) {
+PagerStatus Pager::append(long long frame_idx, int mode, int* page, int* special_slot) {
   if (pending_ || frame_idx <= last_frame_) return PagerStatus::kSequence;
-  if (is_keyframe && committed_ >= max_frames_) return PagerStatus::kCapacity;
+  if (mode == 1 && committed_ >= max_frames_) return PagerStatus::kCapacity;
   // There is always a free page here: at most scale_frames + sliding_window are held
   // between frames, and P = scale_frames + sliding_window + 1.
   pending_page_ = free_.back();
   free_.pop_back();
   pending_ = true;
-  pending_key_ = is_keyframe;
+  pending_key_ = mode == 1;
+  deferred_ = mode == LBM_KEYFRAME_DEFERRED;
+  attended_ = false;
   pending_frame_ = frame_idx;
   last_frame_ = frame_idx;
   *page = pending_page_;
@@ -70,7 +74,23 @@ PagerStatus Pager::visible(std::vector<int>* pages, int* n_special, int* last_pa
 }
 
 PagerStatus Pager::finish(int* evicted) {
-  if (!pending_) return PagerStatus::kSequence;
+  if (!pending_ || attended_) return PagerStatus::kSequence;
+  *evicted = -1;
+  if (deferred_) {
+    attended_ = true;  // the decision comes with commit()
+    return PagerStatus::kOk;
+  }
+  return settle(evicted);
+}
+
+PagerStatus Pager::commit(bool keep, int* evicted) {
+  if (!pending_ || !deferred_ || !attended_) return PagerStatus::kSequence;
+  if (keep && committed_ >= max_frames_) return PagerStatus::kCapacity;
+  pending_key_ = keep;
+  return settle(evicted);
+}
+
+PagerStatus Pager::settle(int* evicted) {
   *evicted = -1;
   if (pending_key_) {
     const PageEntry e{pending_page_, pending_frame_};
@@ -92,6 +112,8 @@ PagerStatus Pager::finish(int* evicted) {
   pending_ = false;
   pending_page_ = -1;
   pending_key_ = false;
+  deferred_ = false;
+  attended_ = false;
   pending_frame_ = -1;
   return PagerStatus::kOk;
 }
@@ -131,7 +153,8 @@ int fill_state(const Pager& p, lbm_cache_state_t* st) {
       st->special_pages ? p.n_special() - kSpecialPage * (st->special_pages - 1) : 0;
   st->pending = p.pending() ? 1 : 0;
   st->pending_page = p.pending_page();
-  st->pending_is_keyframe = p.pending_is_keyframe() ? 1 : 0;
+  st->pending_is_keyframe = p.pending_deferred() ? LBM_KEYFRAME_DEFERRED
+                                                 : (p.pending_is_keyframe() ? 1 : 0);
   st->pending_frame = p.pending_frame();
   st->last_frame = p.last_frame();
   if (cap < 0) return LBM_ERR_INVALID;
@@ -172,7 +195,8 @@ int lbm_pager_create(int scale_frames, int sliding_window, int max_frames,
 int lbm_pager_append(lbm_pager_t* pager, long long frame_idx, int is_keyframe, int* page,
                      int* special_slot) {
   if (!pager || !page || !special_slot) return LBM_ERR_INVALID;
-  return to_status(pager->p.append(frame_idx, is_keyframe != 0, page, special_slot));
+  if (is_keyframe < 0 || is_keyframe > LBM_KEYFRAME_DEFERRED) return LBM_ERR_INVALID;
+  return to_status(pager->p.append(frame_idx, is_keyframe, page, special_slot));
 }
 
 int lbm_pager_visible(const lbm_pager_t* pager, int* pages, int capacity, int* n_pages,
@@ -192,6 +216,11 @@ int lbm_pager_visible(const lbm_pager_t* pager, int* pages, int capacity, int* n
 int lbm_pager_finish(lbm_pager_t* pager, int* evicted) {
   if (!pager || !evicted) return LBM_ERR_INVALID;
   return to_status(pager->p.finish(evicted));
+}
+
+int lbm_pager_commit(lbm_pager_t* pager, int keep, int* evicted) {
+  if (!pager || !evicted) return LBM_ERR_INVALID;
+  return to_status(pager->p.commit(keep != 0, evicted));
 }
 
 int lbm_pager_reset(lbm_pager_t* pager) {

@@ -4,7 +4,8 @@
 // scale_frames committed keyframes keep their pages, later ones enter a sliding window of
 // sliding_window pages whose oldest page returns to the free list when it overflows.  The
 // special stream is append-only.  [KVBenefits] "Dynamic Keyframe Selection": a frame is
-// placed tentatively, attends, and is then kept (deferred eviction) or rolled back.
+// placed tentatively, attends, and is then kept (deferred eviction) or rolled back -- decided
+// at append, or after the attention when the frame is appended undecided.
 #pragma once
 
 #include <cstdint>
@@ -32,18 +33,25 @@ class Pager {
   void reset();
 
   // Pops a page for frame_idx and reserves the next specials_per_frame special slots.
-  PagerStatus append(long long frame_idx, bool is_keyframe, int* page, int* special_slot);
+  // mode: 0 drop after attention, 1 keep, LBM_KEYFRAME_DEFERRED decide with commit().
+  PagerStatus append(long long frame_idx, int mode, int* page, int* special_slot);
   // What append would return, without changing any state.
-  PagerStatus peek_append(long long frame_idx, bool is_keyframe, int* page,
-                          int* special_slot) const;
+  PagerStatus peek_append(long long frame_idx, int mode, int* page, int* special_slot) const;
   // Visible patch pages of the pending frame, in scale -> window -> own order.
   PagerStatus visible(std::vector<int>* pages, int* n_special, int* last_page_len) const;
-  // Commit or roll back the pending frame; *evicted = page freed by deferred eviction or -1.
+  // After the pending frame's attention: commit or roll back a decided frame (*evicted =
+  // page freed by deferred eviction or -1); an undecided frame only becomes attended.
   PagerStatus finish(int* evicted);
+  // Keep or drop an undecided frame after its attention (kCapacity: keeping it would exceed
+  // max_frames; the frame stays pending).
+  PagerStatus commit(bool keep, int* evicted);
+  // True while a pending frame can still be attended.
+  bool awaiting_attention() const { return pending_ && !attended_; }
 
   bool pending() const { return pending_; }
   int pending_page() const { return pending_page_; }
   bool pending_is_keyframe() const { return pending_key_; }
+  bool pending_deferred() const { return pending_ && deferred_; }
   long long pending_frame() const { return pending_frame_; }
   long long last_frame() const { return last_frame_; }
   int n_special() const { return n_special_; }
@@ -62,8 +70,12 @@ class Pager {
   bool pending_ = false;
   int pending_page_ = -1;
   bool pending_key_ = false;
+  bool deferred_ = false;   // the pending frame waits for commit()
+  bool attended_ = false;   // ... and its attention has been issued
   long long pending_frame_ = -1;
   long long last_frame_ = -1;
+
+  PagerStatus settle(int* evicted);  // commit / roll back the pending frame by pending_key_
 };
 
 // Fills the counts and, where the caller gave room, the arrays of a state snapshot.

@@ -89,8 +89,11 @@ def regen_source(cfg: workloads.StreamConfig, frame_ids: list):
 
 
 def run_stream(cfg: workloads.StreamConfig, check_frames=None, rows=None, frame_ids=None,
-               tamper=None, check_pools=True, regenerate=False, report=None):
+               tamper=None, check_pools=True, regenerate=False, report=None, decide_after=False):
     """Streams every frame of cfg through the cache; checks the frames in check_frames.
+
+    decide_after: append every frame undecided and keep / drop it after its attention
+    (lbm_commit_frame) by the schedule; the oracle takes the same decision at append.
 
     frame_ids: absolute frame index of each streamed frame (default 0..n-1).
     tamper(n, q, k, v) -> (q, k, v): changes the seeded inputs of frame n (stress tests).
@@ -113,8 +116,12 @@ def run_stream(cfg: workloads.StreamConfig, check_frames=None, rows=None, frame_
             q, k, v = tamper(n, q, k, v)
         qd, kd, vd = dev(q, cfg.dtype), dev(k, cfg.dtype), dev(v, cfg.dtype)
         out = torch.empty_like(qd)
-        cache.append_frame(qd, kd, vd, fid, keys[n])
+        cache.append_frame(qd, kd, vd, fid, None if decide_after else keys[n])
         cache.attend_frame(qd, out)
+        if decide_after:
+            st = cache.state()
+            assert st["pending"] and st["pending_is_keyframe"] is None, fid
+            cache.commit_frame(keys[n])
         checking = n in check
         r = so.step(fid, keys[n], q, k, v, rows=rows if checking else [], attend=checking)
         if not checking:

@@ -112,6 +112,64 @@ def test_pager_errors_leave_state_unchanged(lib):
     assert pg.state()["free"] == [3, 2, 1, 0]
 
 
+def test_pager_decisions_after_attention_replay_bit_exactly(lib):
+    """Frames appended undecided (LBM_KEYFRAME_DEFERRED), attended, then kept or dropped
+    give the page table the oracle gives for the same decisions."""
+    rng = np.random.default_rng(5)
+    for _ in range(20):
+        S, W = int(rng.integers(0, 5)), int(rng.integers(0, 7))
+        n = int(rng.integers(1, 90))
+        sched = [bool(x) for x in rng.random(n) < rng.uniform(0.1, 1.0)]
+        pg = _lib.Pager(S, W, max(1, sum(sched)))
+        orc = retention.PagedRetention(S, W, max(1, sum(sched)))
+        for f, key in enumerate(sched):
+            assert pg.append(f, None) == orc.append(f, None)
+            pages, n_sp, last = pg.visible()
+            assert pages == orc.visible().patch_pages
+            assert pg.finish() == -1                    # attended, still undecided
+            st = pg.state()
+            assert st["pending"] and st["pending_is_keyframe"] is None
+            oev = orc.finish(keep=key)
+            assert pg.commit(key) == (-1 if oev is None else oev)
+            st, snap = pg.state(), orc.snapshot()
+            for k in ("scale_pages", "scale_frames", "window_pages", "window_frames", "free",
+                      "n_special"):
+                assert st[k] == snap[k], (f, k)
+            assert not st["pending"]
+        pg.close()
+
+
+def test_pager_decision_after_attention_errors(lib):
+    pg = _lib.Pager(1, 1, 2)
+    page, slot = ctypes.c_int(), ctypes.c_int()
+    assert lib.lbm_pager_append(pg.handle, 0, 3, ctypes.byref(page),
+                                ctypes.byref(slot)) == _lib.LBM_ERR_INVALID  # not 0, 1, 2
+    pg.append(0, None)
+    with pytest.raises(_lib.LbmError) as e:
+        pg.commit(True)                             # not attended yet
+    assert e.value.status == _lib.LBM_ERR_SEQUENCE
+    pg.finish()
+    with pytest.raises(_lib.LbmError) as e:
+        pg.finish()                                 # attended twice
+    assert e.value.status == _lib.LBM_ERR_SEQUENCE
+    pg.commit(True)
+    pg.append(1, True)
+    pg.finish()
+    with pytest.raises(_lib.LbmError) as e:
+        pg.commit(True)                             # decided at append, already settled
+    assert e.value.status == _lib.LBM_ERR_SEQUENCE
+    pg.append(2, None)
+    pg.finish()
+    before = pg.state()
+    with pytest.raises(_lib.LbmError) as e:
+        pg.commit(True)                             # max_frames = 2 keyframes already kept
+    assert e.value.status == _lib.LBM_ERR_CAPACITY
+    assert pg.state() == before                     # still pending
+    pg.commit(False)
+    assert not pg.state()["pending"]
+    pg.close()
+
+
 def test_create_argument_checks_without_gpu(lib):
     h = ctypes.c_void_p()
     # pager: bad sizes

@@ -75,6 +75,13 @@ def test_forced_grid_sizes_agree(grid, monkeypatch):
     run_stream(custom_config(205, 2, 64, "bf16", 12, 12, 8, 1, 2, 3))
 
 
+def test_keyframes_decided_after_attention():
+    """[KVBenefits] "Dynamic Keyframe Selection": each frame is appended undecided, attends,
+    and is then kept or dropped (every 3rd kept); outputs, pages and page table match the
+    oracle that took the same decisions at append."""
+    run_stream(custom_config(210, 2, 64, "bf16", 6, 9, 14, 3, 1, 2), decide_after=True)
+
+
 def test_non_contiguous_frame_indices():
     cfg = custom_config(206, 2, 64, "bf16", 5, 7, 8, 2, 1, 2)
     run_stream(cfg, frame_ids=[0, 3, 4, 10, 11, 20, 57, 58])
@@ -171,6 +178,17 @@ def test_sequence_errors_leave_state_unchanged():
     cache.reset()
     st = cache.state()
     assert st["free"] == [2, 1, 0] and st["n_special"] == 0 and not st["pending"]
+    cache.append_frame(q, k, v, 0, None)                  # decided after attention
+    with pytest.raises(_lib.LbmError) as e:
+        cache.commit_frame(True)                          # not attended yet
+    assert e.value.status == _lib.LBM_ERR_SEQUENCE
+    cache.attend_frame(q, out)
+    with pytest.raises(_lib.LbmError) as e:
+        cache.attend_frame(q, out)                        # attended, still undecided
+    assert e.value.status == _lib.LBM_ERR_SEQUENCE
+    cache.commit_frame(True)
+    assert cache.state()["scale_frames"] == [0] and not cache.state()["pending"]
+    cache.check()
     with pytest.raises(_lib.LbmError) as e:
         _lib.PagedKVCache(rope, 2, 96, 16, 1, 1, 2, _lib.LBM_BF16)
     assert e.value.status == _lib.LBM_ERR_UNSUPPORTED

@@ -163,3 +163,44 @@ def test_sequence_and_capacity_errors():
         r.append(4, True)
     r.append(4, False)          # non-keyframes still fit
     r.finish()
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_decision_after_attention_equals_decision_at_append(seed):
+    """"Dynamic Keyframe Selection": keeping or dropping a frame after its attention gives
+    the state the same decision taken at append gives, frame by frame, and the retained set
+    of the closed form."""
+    rng = np.random.default_rng(seed)
+    S, W = int(rng.integers(0, 5)), int(rng.integers(0, 7))
+    n = int(rng.integers(5, 80))
+    sched = [bool(x) for x in rng.random(n) < rng.uniform(0.2, 0.9)]
+    up_front = retention.PagedRetention(S, W, max(1, sum(sched)))
+    deferred = retention.PagedRetention(S, W, max(1, sum(sched)))
+    committed = []
+    for f, key in enumerate(sched):
+        assert up_front.append(f, key) == deferred.append(f, None)
+        assert up_front.visible() == deferred.visible()
+        assert up_front.finish() == deferred.finish(keep=key)
+        assert up_front.snapshot() == deferred.snapshot()
+        if key:
+            committed.append(f)
+        assert deferred.retained_frames() == retention.retained_closed_form(committed, S, W)
+
+
+def test_decision_after_attention_errors():
+    r = retention.PagedRetention(1, 1, 1)
+    r.append(0, None)
+    with pytest.raises(retention.SequenceError):
+        r.finish()                              # undecided frame needs keep
+    r.finish(keep=True)
+    r.append(1, False)
+    with pytest.raises(retention.SequenceError):
+        r.finish(keep=True)                     # decided at append: no second decision
+    r.finish()
+    r.append(2, None)
+    before = r.snapshot()
+    with pytest.raises(retention.CapacityError):
+        r.finish(keep=True)                     # max_frames = 1 keyframe already kept
+    assert r.snapshot() == before               # still pending, unchanged
+    r.finish(keep=False)
+    assert r.snapshot()["pending"] is None
