@@ -91,6 +91,16 @@ LBM_API int lbm_rope3d_tables(int head_dim, int ppf, int pph, int ppw, int patch
 /* Writes the expanded table of [3DRoPE-KV] "Multi-Axis Frequency Generation": cos and sin,
  * each float [ppf * (patch_start_idx + pph*ppw)][head_dim/2] (device pointers, caller-owned),
  * frames 0..ppf-1 in order, tokens of a frame in the order above.  Enqueued on stream. */
+/* The same tables with an explicit (t, h, w) split of head_dim = d_t + d_h + d_w (the pages'
+ * fhw_dim, e.g. [20, 22, 22] for head_dim 64 in [3DRoPE-KV] "Implementation Example" and
+ * [40, 44, 44] for 128 in [VideoRoPE] "Enabling 3D RoPE for Video Heads") and an NTK factor
+ * that multiplies theta ([VideoRoPE] "NTK-Aware Frequency Scaling").  Each axis size even and
+ * >= 2, ntk_factor > 0, theta * ntk_factor > 1; otherwise LBM_ERR_INVALID.  lbm_rope3d_tables
+ * is this call with the default split and ntk_factor 1. */
+LBM_API int lbm_rope3d_tables_fhw(int d_t, int d_h, int d_w, int ppf, int pph, int ppw,
+                                  int patch_start_idx, double theta, double ntk_factor,
+                                  lbm_rope_t** out);
+
 LBM_API int lbm_rope3d_expand(const lbm_rope_t* rope, float* cos_out, float* sin_out, void* stream);
 
 LBM_API void lbm_rope_destroy(lbm_rope_t* rope);

@@ -12,7 +12,11 @@ What the pages fix
   multiplication written in real arithmetic.
 * [VideoRoPE] "The Three Rotary Dimensions" and "NTK-Aware Frequency Scaling": the 1D
   table of an axis is built from ``theta`` (10000) and an ``ntk_factor`` that multiplies
-  theta (fixed at 1 here).
+  theta (1 unless given).
+* [3DRoPE-KV] "Implementation Example" and [VideoRoPE] "Enabling 3D RoPE for Video Heads"
+  print explicit (t, h, w) feature splits ``fhw_dim`` = [20, 22, 22] (head_dim 64) and
+  [40, 44, 44] (head_dim 128); every function below takes such a ``split`` instead of the
+  default one.
 * [VideoRoPE] "Temporal Consistency in KV-Cache Streaming": the t coordinate is the
   absolute (global) frame index of the stream.
 
@@ -33,10 +37,18 @@ import numpy as np
 THETA = 10000.0
 
 
-def axis_split(head_dim: int) -> tuple[int, int, int]:
-    """Feature counts (d_t, d_h, d_w) of the three axes; all even, summing to head_dim."""
+def axis_split(head_dim: int, split=None) -> tuple[int, int, int]:
+    """Feature counts (d_t, d_h, d_w) of the three axes; all even, summing to head_dim.
+
+    ``split`` gives them explicitly (the pages' ``fhw_dim``); otherwise the default reading.
+    """
     if head_dim % 2 != 0 or head_dim < 6:
         raise ValueError("head_dim must be even and >= 6")
+    if split is not None:
+        d_t, d_h, d_w = (int(x) for x in split)
+        if d_t + d_h + d_w != head_dim or min(d_t, d_h, d_w) < 2 or d_t % 2 or d_h % 2 or d_w % 2:
+            raise ValueError("split must be three even sizes >= 2 summing to head_dim")
+        return d_t, d_h, d_w
     d_h = 2 * (head_dim // 6)
     d_w = d_h
     d_t = head_dim - d_h - d_w
@@ -53,15 +65,16 @@ def inv_freq(d_axis: int, theta: float = THETA, ntk_factor: float = 1.0) -> np.n
     return base ** (-(2.0 * i) / float(d_axis))
 
 
-def axis_tables(head_dim: int, n_t: int, n_h: int, n_w: int, theta: float = THETA):
+def axis_tables(head_dim: int, n_t: int, n_h: int, n_w: int, theta: float = THETA,
+                split=None, ntk_factor: float = 1.0):
     """Per-axis angle tables: ang_t[n_t, d_t/2], ang_h[n_h, d_h/2], ang_w[n_w, d_w/2].
 
     Row p of an axis table holds p * inv_freq of that axis (fp64 angles in radians).
     """
-    d_t, d_h, d_w = axis_split(head_dim)
-    ang_t = np.outer(np.arange(n_t, dtype=np.float64), inv_freq(d_t, theta))
-    ang_h = np.outer(np.arange(n_h, dtype=np.float64), inv_freq(d_h, theta))
-    ang_w = np.outer(np.arange(n_w, dtype=np.float64), inv_freq(d_w, theta))
+    d_t, d_h, d_w = axis_split(head_dim, split)
+    ang_t = np.outer(np.arange(n_t, dtype=np.float64), inv_freq(d_t, theta, ntk_factor))
+    ang_h = np.outer(np.arange(n_h, dtype=np.float64), inv_freq(d_h, theta, ntk_factor))
+    ang_w = np.outer(np.arange(n_w, dtype=np.float64), inv_freq(d_w, theta, ntk_factor))
     return ang_t, ang_h, ang_w
 
 
@@ -79,22 +92,23 @@ def token_positions(frame_idx: int, patch_start_idx: int, pph: int, ppw: int) ->
     return pos
 
 
-def angles_for_positions(pos: np.ndarray, head_dim: int, theta: float = THETA) -> np.ndarray:
+def angles_for_positions(pos: np.ndarray, head_dim: int, theta: float = THETA, split=None,
+                         ntk_factor: float = 1.0) -> np.ndarray:
     """Rotation angle of every (token, pair): [N, head_dim/2] fp64, pairs ordered t, h, w."""
-    d_t, d_h, d_w = axis_split(head_dim)
+    d_t, d_h, d_w = axis_split(head_dim, split)
     pos = np.asarray(pos, dtype=np.float64)
     return np.concatenate(
         [
-            np.outer(pos[:, 0], inv_freq(d_t, theta)),
-            np.outer(pos[:, 1], inv_freq(d_h, theta)),
-            np.outer(pos[:, 2], inv_freq(d_w, theta)),
+            np.outer(pos[:, 0], inv_freq(d_t, theta, ntk_factor)),
+            np.outer(pos[:, 1], inv_freq(d_h, theta, ntk_factor)),
+            np.outer(pos[:, 2], inv_freq(d_w, theta, ntk_factor)),
         ],
         axis=1,
     )
 
 
 def expanded_table(head_dim: int, ppf: int, pph: int, ppw: int, patch_start_idx: int,
-                   theta: float = THETA, f_start: int = 0):
+                   theta: float = THETA, f_start: int = 0, split=None, ntk_factor: float = 1.0):
     """The concatenated, expanded table as (cos, sin), each [ppf*(psi+pph*ppw), head_dim/2].
 
     Frames f_start .. f_start+ppf-1, each frame's tokens in the order of token_positions.
@@ -103,7 +117,7 @@ def expanded_table(head_dim: int, ppf: int, pph: int, ppw: int, patch_start_idx:
     pos = np.concatenate(
         [token_positions(f_start + f, patch_start_idx, pph, ppw) for f in range(ppf)], axis=0
     )
-    ang = angles_for_positions(pos, head_dim, theta)
+    ang = angles_for_positions(pos, head_dim, theta, split, ntk_factor)
     return np.cos(ang), np.sin(ang)
 
 
@@ -125,8 +139,8 @@ def rotate(x: np.ndarray, angles: np.ndarray) -> np.ndarray:
 
 
 def rotate_frame(x: np.ndarray, frame_idx: int, patch_start_idx: int, pph: int, ppw: int,
-                 theta: float = THETA) -> np.ndarray:
+                 theta: float = THETA, split=None, ntk_factor: float = 1.0) -> np.ndarray:
     """Rotate one frame's tokens x [psi + pph*ppw, H, D] at their 3D positions."""
     head_dim = x.shape[-1]
     pos = token_positions(frame_idx, patch_start_idx, pph, ppw)
-    return rotate(x, angles_for_positions(pos, head_dim, theta))
+    return rotate(x, angles_for_positions(pos, head_dim, theta, split, ntk_factor))

@@ -47,8 +47,10 @@ class FrameResult:
 class StreamOracle:
     def __init__(self, heads: int, head_dim: int, pph: int, ppw: int, scale_frames: int,
                  sliding_window: int, max_frames: int, specials_per_frame: int = 6,
-                 theta: float = rope3d.THETA, keep_history: bool = False, kv_source=None):
-        """kv_source, if given, is a callable (frame, region) -> (k, v) returning a past
+                 theta: float = rope3d.THETA, keep_history: bool = False, kv_source=None,
+                 split=None, ntk_factor: float = 1.0):
+        """split / ntk_factor: an explicit (t, h, w) feature split and NTK factor of the 3D
+        RoPE (``rope3d.axis_split``, ``rope3d.inv_freq``).  kv_source, if given, is a callable (frame, region) -> (k, v) returning a past
         frame's unrotated inputs (region "patch": [pph*ppw, H, D], "special": [6, H, D]);
         the oracle then keeps no K/V of its own and re-creates retained keys when a frame
         attends, which keeps long streams small in memory."""
@@ -58,6 +60,8 @@ class StreamOracle:
         self.ppw = ppw
         self.psi = specials_per_frame
         self.theta = theta
+        self.split = split
+        self.ntk_factor = ntk_factor
         self.ret = retention.PagedRetention(scale_frames, sliding_window, max_frames,
                                             specials_per_frame)
         self.patch_kv: dict = {}      # frame -> (k [Pf,H,D], v [Pf,H,D]) of retained frames
@@ -88,7 +92,8 @@ class StreamOracle:
         k, v = self.kv_source(frame, region)
         pos = rope3d.token_positions(frame, self.psi, self.pph, self.ppw)
         pos = pos[self.psi:] if region == "patch" else pos[:self.psi]
-        kr = rope3d.rotate(k, rope3d.angles_for_positions(pos, self.head_dim, self.theta))
+        kr = rope3d.rotate(k, rope3d.angles_for_positions(pos, self.head_dim, self.theta,
+                                                                self.split, self.ntk_factor))
         return kr, np.asarray(v, dtype=np.float64)
 
     def step(self, frame_idx: int, is_keyframe: bool, q: np.ndarray, k: np.ndarray,
@@ -96,8 +101,10 @@ class StreamOracle:
         T = self.tokens_per_frame
         assert q.shape == (T, self.heads, self.head_dim), q.shape
         page, slot = self.ret.append(frame_idx, is_keyframe)
-        qr = rope3d.rotate_frame(q, frame_idx, self.psi, self.pph, self.ppw, self.theta)
-        kr = rope3d.rotate_frame(k, frame_idx, self.psi, self.pph, self.ppw, self.theta)
+        qr = rope3d.rotate_frame(q, frame_idx, self.psi, self.pph, self.ppw, self.theta,
+                                 self.split, self.ntk_factor)
+        kr = rope3d.rotate_frame(k, frame_idx, self.psi, self.pph, self.ppw, self.theta,
+                                 self.split, self.ntk_factor)
         v64 = np.asarray(v, dtype=np.float64)
         vis = self.ret.visible()
 

@@ -165,12 +165,24 @@ int lbm_rope3d_tables(int head_dim, int ppf, int pph, int ppw, int patch_start_i
                       double theta, lbm_rope_t** out) {
   if (!out) return LBM_ERR_INVALID;
   *out = nullptr;
-  if (head_dim < 6 || head_dim % 2 || ppf < 1 || pph < 1 || ppw < 1 || patch_start_idx < 0 ||
-      !(theta > 1.0) || (long long)pph * ppw > (1 << 20) || ppf > (1 << 24))
-    return LBM_ERR_INVALID;
+  if (head_dim < 6 || head_dim % 2) return LBM_ERR_INVALID;
   // Axis split: d_h = d_w = 2 * (head_dim / 6), d_t = the rest; pairs ordered t, h, w.
   const int dh = 2 * (head_dim / 6);
-  const int dt = head_dim - 2 * dh;
+  return lbm_rope3d_tables_fhw(head_dim - 2 * dh, dh, dh, ppf, pph, ppw, patch_start_idx, theta,
+                               1.0, out);
+}
+
+int lbm_rope3d_tables_fhw(int dt, int dh, int dw, int ppf, int pph, int ppw,
+                          int patch_start_idx, double theta, double ntk_factor,
+                          lbm_rope_t** out) {
+  if (!out) return LBM_ERR_INVALID;
+  *out = nullptr;
+  if (dt < 2 || dh < 2 || dw < 2 || dt % 2 || dh % 2 || dw % 2 || ppf < 1 || pph < 1 ||
+      ppw < 1 || patch_start_idx < 0 || !(ntk_factor > 0.0) || !(theta * ntk_factor > 1.0) ||
+      (long long)pph * ppw > (1 << 20) || ppf > (1 << 24))
+    return LBM_ERR_INVALID;
+  const int head_dim = dt + dh + dw;
+  theta *= ntk_factor;  // [VideoRoPE] "NTK-Aware Frequency Scaling": theta * ntk_factor
   lbm::RopeTables t{};
   t.head_dim = head_dim;
   t.ppf = ppf;
@@ -179,7 +191,7 @@ int lbm_rope3d_tables(int head_dim, int ppf, int pph, int ppw, int patch_start_i
   t.psi = patch_start_idx;
   t.nt = dt / 2;
   t.nh = dh / 2;
-  t.nw = dh / 2;
+  t.nw = dw / 2;
   const size_t n_t = (size_t)ppf * t.nt, n_h = (size_t)(pph + 1) * t.nh,
                n_w = (size_t)(ppw + 1) * t.nw;
   std::vector<float2> host(n_t + n_h + n_w);
@@ -195,7 +207,7 @@ int lbm_rope3d_tables(int head_dim, int ppf, int pph, int ppw, int patch_start_i
   };
   fill(host.data(), ppf, t.nt, dt);
   fill(host.data() + n_t, pph + 1, t.nh, dh);
-  fill(host.data() + n_t + n_h, ppw + 1, t.nw, dh);
+  fill(host.data() + n_t + n_h, ppw + 1, t.nw, dw);
   auto* r = new (std::nothrow) lbm_rope;
   if (!r) return LBM_ERR_NOMEM;
   if (cudaGetDevice(&r->device) != cudaSuccess ||

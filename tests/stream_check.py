@@ -64,9 +64,10 @@ def check_attn(got: np.ndarray, exact: np.ndarray, what: str) -> tuple[float, fl
     return rel, mx
 
 
-def make_cache(cfg: workloads.StreamConfig, max_frame_idx: int | None = None):
+def make_cache(cfg: workloads.StreamConfig, max_frame_idx: int | None = None, split=None,
+               ntk_factor: float = 1.0):
     ppf = (max_frame_idx + 1) if max_frame_idx is not None else cfg.n_frames
-    rope = _lib.Rope3D(cfg.head_dim, ppf, cfg.pph, cfg.ppw, 6)
+    rope = _lib.Rope3D(cfg.head_dim, ppf, cfg.pph, cfg.ppw, 6, split=split, ntk_factor=ntk_factor)
     cache = _lib.PagedKVCache(rope, cfg.heads, cfg.head_dim, cfg.patches, cfg.scale_frames,
                               cfg.sliding_window, max(1, cfg.n_keyframes),
                               _lib.LBM_BF16 if cfg.dtype == "bf16" else _lib.LBM_F32)
@@ -89,9 +90,13 @@ def regen_source(cfg: workloads.StreamConfig, frame_ids: list):
 
 
 def run_stream(cfg: workloads.StreamConfig, check_frames=None, rows=None, frame_ids=None,
-               tamper=None, check_pools=True, regenerate=False, report=None, decide_after=False):
+               tamper=None, check_pools=True, regenerate=False, report=None, decide_after=False,
+               split=None, ntk_factor: float = 1.0, reset_at=()):
     """Streams every frame of cfg through the cache; checks the frames in check_frames.
 
+    split, ntk_factor: RoPE variant (explicit (t, h, w) split, NTK factor), for both sides.
+    reset_at: stream positions before which cache and oracle are reset (windowed streaming;
+    frame_ids may then start again).
     decide_after: append every frame undecided and keep / drop it after its attention
     (lbm_commit_frame) by the schedule; the oracle takes the same decision at append.
 
@@ -103,14 +108,18 @@ def run_stream(cfg: workloads.StreamConfig, check_frames=None, rows=None, frame_
     import torch
     frame_ids = list(range(cfg.n_frames)) if frame_ids is None else list(frame_ids)
     check = set(range(cfg.n_frames)) if check_frames is None else set(check_frames)
-    rope, cache = make_cache(cfg, max(frame_ids))
+    rope, cache = make_cache(cfg, max(frame_ids), split, ntk_factor)
     so = ostream.StreamOracle(cfg.heads, cfg.head_dim, cfg.pph, cfg.ppw, cfg.scale_frames,
                               cfg.sliding_window, max(1, cfg.n_keyframes),
-                              kv_source=regen_source(cfg, frame_ids) if regenerate else None)
+                              kv_source=regen_source(cfg, frame_ids) if regenerate else None,
+                              split=split, ntk_factor=ntk_factor)
     summary = []
     T = cfg.tokens
     keys = cfg.keyframes
     for n, fid in enumerate(frame_ids):
+        if n in reset_at:
+            cache.reset()
+            so.reset()
         q, k, v = workloads.frame_qkv(cfg, n)
         if tamper is not None:
             q, k, v = tamper(n, q, k, v)

@@ -170,6 +170,17 @@ def test_pager_decision_after_attention_errors(lib):
     pg.close()
 
 
+def test_rope_variant_argument_checks_without_gpu(lib):
+    h = ctypes.c_void_p()
+    for args in [(20, 22, 21), (0, 32, 32), (21, 21, 22)]:          # odd or empty axes
+        assert lib.lbm_rope3d_tables_fhw(*args, 4, 3, 3, 6, 10000.0, 1.0,
+                                         ctypes.byref(h)) == _lib.LBM_ERR_INVALID
+    assert lib.lbm_rope3d_tables_fhw(20, 22, 22, 4, 3, 3, 6, 10000.0, 0.0,
+                                     ctypes.byref(h)) == _lib.LBM_ERR_INVALID   # ntk <= 0
+    assert lib.lbm_rope3d_tables_fhw(20, 22, 22, 4, 3, 3, 6, 1.0, 0.5,
+                                     ctypes.byref(h)) == _lib.LBM_ERR_INVALID   # theta*ntk <= 1
+
+
 def test_create_argument_checks_without_gpu(lib):
     h = ctypes.c_void_p()
     # pager: bad sizes

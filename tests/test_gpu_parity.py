@@ -45,6 +45,31 @@ def test_rope_tables_match_oracle(head_dim, ppf, pph, ppw):
     rope.close()
 
 
+@pytest.mark.parametrize("head_dim,split,ntk", [(64, (20, 22, 22), 1.0), (128, (40, 44, 44), 4.0),
+                                                (64, None, 2.0)])
+def test_rope_variant_tables_match_oracle(head_dim, split, ntk):
+    """Explicit (t, h, w) splits as printed on the pages, and the NTK factor."""
+    import torch
+    rope = _lib.Rope3D(head_dim, 12, 9, 11, 6, split=split, ntk_factor=ntk)
+    rows = 12 * (6 + 9 * 11)
+    cos = torch.empty(rows, head_dim // 2, device="cuda")
+    sin = torch.empty_like(cos)
+    rope.expand(cos, sin)
+    torch.cuda.synchronize()
+    ec, es = rope3d.expanded_table(head_dim, 12, 9, 11, 6, split=split, ntk_factor=ntk)
+    assert np.abs(cos.cpu().numpy() - ec).max() <= 1e-5
+    assert np.abs(sin.cpu().numpy() - es).max() <= 1e-5
+    rope.close()
+
+
+@pytest.mark.parametrize("head_dim,split,ntk", [(64, (20, 22, 22), 1.0), (128, (40, 44, 44), 4.0)])
+def test_rope_variant_stream(head_dim, split, ntk):
+    """Fused rotate + append and attention with a RoPE variant: q, pages and outputs match
+    the oracle rotating with the same split and NTK factor."""
+    run_stream(custom_config(211 + head_dim // 64, 2, head_dim, "bf16", 5, 8, 7, 2, 1, 2),
+               split=split, ntk_factor=ntk)
+
+
 def test_tiny_fp32_config_all_frames():
     run_stream(CONFIGS[0])
 
@@ -80,6 +105,15 @@ def test_keyframes_decided_after_attention():
     and is then kept or dropped (every 3rd kept); outputs, pages and page table match the
     oracle that took the same decisions at append."""
     run_stream(custom_config(210, 2, 64, "bf16", 6, 9, 14, 3, 1, 2), decide_after=True)
+
+
+def test_windowed_stream_resets_between_windows():
+    """[KVBenefits] "Cross-Window Alignment for Long Videos": a long video processed in
+    windows, the cache cleaned (lbm_cache_reset) before each window and frame indices
+    starting again at 0: every window matches a fresh oracle, so nothing of an earlier window
+    (pages, special tokens) stays visible."""
+    cfg = custom_config(214, 2, 64, "bf16", 6, 7, 21, 2, 1, 2)
+    run_stream(cfg, frame_ids=list(range(7)) * 3, reset_at=(7, 14))
 
 
 def test_non_contiguous_frame_indices():

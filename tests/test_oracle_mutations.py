@@ -53,7 +53,7 @@ def test_rotate_half_pairing_is_caught(monkeypatch):
         out[..., h:] = x[..., :h] * s + x[..., h:] * c
         return out
     monkeypatch.setattr(rope3d, "rotate", bad_rotate)
-    _fails(tp.test_each_axis_is_library_1d_rope, 64)
+    _fails(tp.test_each_axis_is_library_1d_rope, 64, None, 1.0)
 
 
 def test_transposed_patch_grid_is_caught(monkeypatch):
@@ -102,3 +102,22 @@ def test_specials_not_kept_is_caught(monkeypatch):
         return orig(frames, current, [], retained_before, spf, tpf)
     monkeypatch.setattr(attention, "history_mask", bad_mask)
     _fails(ta.test_stream_two_formulations_agree, ta.CONFIGS[0])
+
+
+def test_ntk_factor_ignored_is_caught(monkeypatch):
+    orig = rope3d.inv_freq
+
+    def bad_inv_freq(d_axis, theta=rope3d.THETA, ntk_factor=1.0):
+        return orig(d_axis, theta, 1.0)
+    monkeypatch.setattr(rope3d, "inv_freq", bad_inv_freq)
+    _fails(tp.test_each_axis_is_library_1d_rope, 64, "example_fhw_dim", 4.0)
+
+
+def test_split_axes_swapped_is_caught(monkeypatch):
+    orig = rope3d.axis_split
+
+    def bad_split(head_dim, split=None):
+        d_t, d_h, d_w = orig(head_dim, split)
+        return d_h, d_t, d_w
+    monkeypatch.setattr(rope3d, "axis_split", bad_split)
+    _fails(tp.test_each_axis_is_library_1d_rope, 64, "example_fhw_dim", 1.0)

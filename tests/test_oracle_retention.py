@@ -204,3 +204,27 @@ def test_decision_after_attention_errors():
     assert r.snapshot() == before               # still pending, unchanged
     r.finish(keep=False)
     assert r.snapshot()["pending"] is None
+
+
+def test_reset_gives_a_fresh_cache():
+    """"Cross-Window Alignment for Long Videos" (clean_kv_cache between windows): after any
+    stream, reset() leaves the state of a new cache, and a second window replays exactly as
+    on a new cache, frame indices starting again at 0."""
+    rng = np.random.default_rng(9)
+    for _ in range(10):
+        S, W = int(rng.integers(0, 4)), int(rng.integers(0, 6))
+        first = [bool(x) for x in rng.random(int(rng.integers(1, 40))) < 0.6]
+        second = [bool(x) for x in rng.random(int(rng.integers(1, 40))) < 0.6]
+        m = max(1, sum(first), sum(second))
+        r = retention.PagedRetention(S, W, m)
+        for f, key in enumerate(first):
+            r.append(f, key)
+            r.finish()
+        r.reset()
+        fresh = retention.PagedRetention(S, W, m)
+        assert r.snapshot() == fresh.snapshot()
+        for f, key in enumerate(second):
+            assert r.append(f, key) == fresh.append(f, key)
+            assert r.visible() == fresh.visible()
+            assert r.finish() == fresh.finish()
+            assert r.snapshot() == fresh.snapshot()

@@ -37,6 +37,14 @@ def test_expanded_table_shape_matches_page_example():
     assert sin.shape == cos.shape
 
 
+def test_page_splits_are_accepted_and_bad_splits_refused():
+    assert rope3d.axis_split(64, _fhw("example_fhw_dim")) == (20, 22, 22)
+    assert rope3d.axis_split(128, _fhw("video_head_fhw_dim")) == (40, 44, 44)
+    for bad in [(20, 22, 20), (21, 21, 22), (0, 32, 32)]:
+        with pytest.raises(ValueError):
+            rope3d.axis_split(64, bad)
+
+
 def test_axis_split_reading():
     # The stated reading: d_h = d_w = 2 * (head_dim // 6), d_t takes the rest.
     assert rope3d.axis_split(64) == (24, 20, 20)
@@ -46,12 +54,12 @@ def test_axis_split_reading():
         assert dt + dh + dw == d and dt % 2 == dh % 2 == dw % 2 == 0 and dh == dw
 
 
-def _llama_rope(d_axis, positions, x_half):
+def _llama_rope(d_axis, positions, x_half, theta=10000.0):
     """transformers' LLaMA rotary embedding of dimension d_axis (rotate-half layout)."""
     from transformers import LlamaConfig
     from transformers.models.llama.modeling_llama import LlamaRotaryEmbedding, apply_rotary_pos_emb
     cfg = LlamaConfig(hidden_size=d_axis * 2, num_attention_heads=2, head_dim=d_axis,
-                      rope_parameters={"rope_type": "default", "rope_theta": 10000.0})
+                      rope_parameters={"rope_type": "default", "rope_theta": theta})
     emb = LlamaRotaryEmbedding(cfg)
     xt = torch.tensor(x_half[None], dtype=torch.float32)        # [1, N, d] -> as [B, H=1?]
     xt = xt[:, None]                                             # [1, 1, N, d]
@@ -74,21 +82,34 @@ def test_inv_freq_matches_library_1d_rope(head_dim):
         np.testing.assert_allclose(ours, lib.double().numpy(), rtol=6e-7, atol=0)   # the library computes in float32
 
 
-@pytest.mark.parametrize("head_dim", [64, 128])
-def test_each_axis_is_library_1d_rope(head_dim):
-    """Features of axis a rotate exactly as a 1D RoPE of dimension d_a at that coordinate."""
+def _fhw(key):
+    return tuple(int(v) for v in _facts()[key].split(","))
+
+
+@pytest.mark.parametrize("head_dim,split,ntk", [(64, None, 1.0), (128, None, 1.0),
+                                                (64, "example_fhw_dim", 1.0),
+                                                (128, "video_head_fhw_dim", 1.0),
+                                                (64, "example_fhw_dim", 4.0),
+                                                (128, None, 2.5)])
+def test_each_axis_is_library_1d_rope(head_dim, split, ntk):
+    """Features of axis a rotate exactly as a 1D RoPE of dimension d_a at that coordinate,
+    with the default split or the pages' explicit fhw_dim splits, and with theta multiplied
+    by ntk_factor ("NTK-Aware Frequency Scaling")."""
     rng = np.random.default_rng(7)
     pph, ppw, psi = 5, 7, 6
     frame = 37
+    split = _fhw(split) if split else None
     x = rng.standard_normal((psi + pph * ppw, 1, head_dim))
-    out = rope3d.rotate_frame(x, frame, psi, pph, ppw)
+    out = rope3d.rotate_frame(x, frame, psi, pph, ppw, split=split, ntk_factor=ntk)
     pos = rope3d.token_positions(frame, psi, pph, ppw)
-    d_t, d_h, d_w = rope3d.axis_split(head_dim)
+    # the axis sizes come from the pages (explicit split) or the stated default reading
+    d_t, d_h, d_w = split if split else {64: (24, 20, 20), 128: (44, 42, 42)}[head_dim]
+    assert sum((d_t, d_h, d_w)) == head_dim
     lo = 0
     for axis, d in enumerate((d_t, d_h, d_w)):
         seg = x[:, 0, lo:lo + d]
         half = np.concatenate([seg[:, 0::2], seg[:, 1::2]], axis=1)   # adjacent -> rotate-half
-        lib = _llama_rope(d, pos[:, axis], half)
+        lib = _llama_rope(d, pos[:, axis], half, theta=10000.0 * ntk)
         back = np.empty_like(seg)
         back[:, 0::2] = lib[:, :d // 2]
         back[:, 1::2] = lib[:, d // 2:]
