@@ -42,9 +42,12 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when max grows by > 2^8
 constexpr unsigned kFull = 0xffffffffu;
 
+constexpr int kMaxStages = 4;  // K/V ring stages the barrier block has room for
+
 template <int D>
 struct Cfg {
   static constexpr int NS = D == 64 ? 4 : 2;            // K/V pipeline stages
+  static_assert(NS <= kMaxStages, "the barrier block holds kMaxStages ring barriers");
   static constexpr int ATOM_BYTES = 128 * 128;          // 128 rows x 64 bf16 (one swizzle atom column)
   static constexpr int ATOMS = D / 64;
   static constexpr int TILE_BYTES = ATOMS * ATOM_BYTES; // one Q, K or V tile
@@ -312,8 +315,8 @@ struct Bars {
   uint64_t pv_done[2];     // per g: PV_j finished (P buffer and O are free again)
   uint64_t o_free[2];      // per g: the epilogue has read O of the segment
   uint64_t drain[2];
-  uint64_t kv_full[4];
-  uint64_t kv_empty[4];    // one arrival per MMA issuer (count 2)
+  uint64_t kv_full[kMaxStages];
+  uint64_t kv_empty[kMaxStages];  // one arrival per MMA issuer (count 2)
   uint32_t tmem_base;
   int abort_flag;
 };
