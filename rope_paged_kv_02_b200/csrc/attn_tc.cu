@@ -781,31 +781,38 @@ __device__ __forceinline__ int last_start_at_or_before(const AttnParams& p, int 
 
 // Merges the partial results of the units that span more than one CTA:
 // out[row][h] = sum_s w_s o_s / sum_s w_s with w_s = 2^(lse_s - max_s lse_s).
-// One warp per (unit, two rows of the pair): each half-warp owns one row, its 16 lanes hold
-// D / 16 features each.  Lane s of a half loads the LSE of segment s (16 at a time), the half
-// reduces max and weights with shuffles, then the O rows of four segments are loaded before
-// any is used, so a row costs about two L2 round trips.
+// One warp per (unit, four rows of the pair): each quarter-warp owns one row, its 8 lanes
+// hold D / 8 features each.  Lane s of a quarter loads the LSE of segment s (8 at a time),
+// the quarter reduces max and weights with shuffles, then the O rows of four segments (two
+// for head_dim 128) are loaded before any is used, so a row costs about two L2 round trips,
+// and the index work of a warp is shared by four rows.  32-bit indices: a frame's partials are far below 2^31
+// floats.
 template <int D>
 __global__ void __launch_bounds__(256) attn_combine_kernel(const __grid_constant__ AttnParams p) {
-  constexpr int VPL = D / 16;  // features per lane
+  constexpr int VPL = D / 8;   // features per lane
   constexpr int V4 = VPL / 4;  // float4 loads per lane and segment
-  const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  constexpr int RPW = 4;       // rows per warp
+  constexpr int SB = D == 64 ? 4 : 2;  // segments whose O rows are loaded before use
+  const unsigned gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  const int half = lane >> 4;
-  const int hl = lane & 15;
-  const long long units = (long long)p.n_pairs * p.heads;
-  if (gw >= units * BM) return;  // BM warps x 2 rows = the 256 rows of a unit
-  const int unit = (int)(gw / BM);
-  const int row_in_pair = (int)(gw - (long long)unit * BM) * 2 + half;
-  const int pair = unit % p.n_pairs;
+  const int quarter = lane >> 3;
+  const int ql = lane & 7;
+  const unsigned units = (unsigned)(p.n_pairs * p.heads);
+  constexpr unsigned kWarpsPerUnit = 2 * BM / RPW;
+  if (gw >= units * kWarpsPerUnit) return;
+  const int unit = (int)(gw / kWarpsPerUnit);
+  const int row_in_pair = (int)(gw - (unsigned)unit * kWarpsPerUnit) * RPW + quarter;
   const int head = unit / p.n_pairs;
+  const int pair = unit - head * p.n_pairs;
   const int row = 2 * pair * BM + row_in_pair;
   const int first = unit * p.n_tiles;
+  const int last = first + p.n_tiles - 1;
   // CTAs whose share [sk_start[c], sk_start[c+1]) meets this unit: c0 .. c1 (the shares are
-  // non-empty and increasing, so c0 and c1 are the last CTAs starting at or before the
-  // unit's first and last item)
+  // non-empty and increasing: c0 is the last CTA starting at or before the unit's first
+  // item, c1 the last starting at or before its last item, a few CTAs after c0)
   const int c0 = last_start_at_or_before(p, first);
-  const int c1 = last_start_at_or_before(p, first + p.n_tiles - 1);
+  int c1 = c0;
+  while (c1 + 1 < p.grid && p.sk_start[c1 + 1] <= last) ++c1;
   if (c1 == c0) return;  // one CTA did the whole unit and wrote the output itself
   // the index arithmetic above reads only kernel parameters and overlapped the attention
   // kernel's tail; its partials are read only after it has completed
@@ -813,37 +820,37 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const __grid_constant
   const bool valid = row < p.tokens;  // rows past the frame have no partials
   const int nseg = c1 - c0 + 1;
   // partial row of segment (CTA c0 + s): slot unit + c
-  auto prow = [&](int s) { return ((long long)unit + c0 + s) * (2 * BM) + row_in_pair; };
+  const int r0 = (unit + c0) * (2 * BM) + row_in_pair;
   float mx = -INFINITY;
-  for (int s0 = 0; s0 < nseg; s0 += 16) {
-    const float v = valid && s0 + hl < nseg ? p.part_lse[prow(s0 + hl)] : -INFINITY;
+  for (int s0 = 0; s0 < nseg; s0 += 8) {
+    const float v = valid && s0 + ql < nseg ? p.part_lse[r0 + (s0 + ql) * (2 * BM)] : -INFINITY;
     mx = fmaxf(mx, v);
   }
 #pragma unroll
-  for (int o = 8; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  for (int o = 4; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   float acc[VPL];
 #pragma unroll
   for (int i = 0; i < VPL; ++i) acc[i] = 0.f;
   float wsum = 0.f;
-  for (int s0 = 0; s0 < nseg; s0 += 16) {
+  for (int s0 = 0; s0 < nseg; s0 += 8) {
     const float w_lane =
-        valid && s0 + hl < nseg ? exp2f(p.part_lse[prow(s0 + hl)] - mx) : 0.f;
-    const int cnt = min(16, nseg - s0);  // the same for both halves (one unit per warp)
-    for (int k0 = 0; k0 < cnt; k0 += 4) {
-      float4 v[4][V4];
-      float w[4];
+        valid && s0 + ql < nseg ? fast_exp2(p.part_lse[r0 + (s0 + ql) * (2 * BM)] - mx) : 0.f;
+    const int cnt = min(8, nseg - s0);  // the same for every quarter (one unit per warp)
+    for (int k0 = 0; k0 < cnt; k0 += SB) {
+      float4 v[SB][V4];
+      float w[SB];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int k = k0 + u;
-        w[u] = __shfl_sync(0xffffffffu, w_lane, (half << 4) + min(k, cnt - 1));
+      for (int u = 0; u < SB; ++u) {
+        const int k = min(k0 + u, cnt - 1);
+        w[u] = __shfl_sync(0xffffffffu, w_lane, (quarter << 3) + k);
         const float4* po = reinterpret_cast<const float4*>(
-            p.part_o + prow(s0 + min(k, cnt - 1)) * D + hl * VPL);
+            p.part_o + (size_t)(r0 + (s0 + k) * (2 * BM)) * D + ql * VPL);
 #pragma unroll
         for (int q = 0; q < V4; ++q)
-          v[u][q] = valid && k < cnt ? po[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+          v[u][q] = valid && k0 + u < cnt ? po[q] : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < SB; ++u) {
         if (k0 + u >= cnt) break;
         wsum += w[u];
 #pragma unroll
@@ -858,8 +865,8 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const __grid_constant
   }
   if (!valid) return;
   const float inv = 1.f / wsum;
-  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + ((long long)row * p.heads + head) * D +
-                     hl * VPL;
+  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + ((size_t)row * p.heads + head) * D +
+                     ql * VPL;
 #pragma unroll
   for (int q = 0; q < V4; ++q)
     *reinterpret_cast<uint2*>(o + 4 * q) =
@@ -924,7 +931,7 @@ cudaError_t launch_attn_tc(const AttnParams& p, int head_dim, cudaStream_t s) {
 }
 
 cudaError_t launch_attn_combine(const AttnParams& p, int head_dim, cudaStream_t s) {
-  const long long warps = (long long)p.n_pairs * p.heads * BM;  // two rows per warp
+  const long long warps = (long long)p.n_pairs * p.heads * (2 * BM / 4);  // four rows a warp
   const dim3 blocks((unsigned)((warps * 32 + 255) / 256));
   if (head_dim == 64) return launch_pdl(attn_combine_kernel<64>, blocks, dim3(256), 0, s, p);
   if (head_dim == 128) return launch_pdl(attn_combine_kernel<128>, blocks, dim3(256), 0, s, p);
