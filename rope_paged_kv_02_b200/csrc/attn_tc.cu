@@ -321,6 +321,8 @@ struct Bars {
   int abort_flag;
 };
 
+static_assert(sizeof(Bars) <= 256, "barrier block exceeds its shared-memory slot");
+
 // Tensor-memory columns of query tile g (256 columns at 256 g): S [0,128); head_dim 64:
 // P [128,192), O [192,256); head_dim 128: O [128,256), P written over S [0,64) after S is
 // read into registers.
