@@ -126,6 +126,21 @@ LBM_API int lbm_cache_create(int heads, int head_dim, int patches_per_frame, int
                      int scale_frames, int sliding_window, int max_frames, int dtype,
                      const lbm_rope_t* rope, lbm_cache_t** out);
 
+/* A cache for num_blocks transformer blocks (1..1024) that share one page table
+ * ([3DRoPE-KV] "Implementation Example": the cache manager is created for num_blocks blocks,
+ * and appending and attention take a block_idx).  Every block has its own K/V pools (the
+ * sizes of lbm_cache_create, times num_blocks) and tensor maps; the page table, free list and
+ * special-stream count are shared, since every block sees the same frames.  A frame visits
+ * the blocks in order: for b = 0 .. num_blocks-1, append (block b) then attend (block b).
+ * Block 0's append takes the frame's page and special slots, later blocks write theirs at the
+ * same places, and the frame is committed or rolled back after the last block's attention.
+ * lbm_cache_create is num_blocks = 1; lbm_append_frame / lbm_attend_frame act on the next
+ * block in that order.  Synchronous. */
+LBM_API int lbm_cache_create_blocks(int num_blocks, int heads, int head_dim,
+                                    int patches_per_frame, int specials_per_frame,
+                                    int scale_frames, int sliding_window, int max_frames,
+                                    int dtype, const lbm_rope_t* rope, lbm_cache_t** out);
+
 /* Rotate and append one frame.  [3DRoPE-KV] "Frame Appending and Position Encoding
  * Integration" and "Complex-Valued Tensor Application"; [VideoRoPE] "Temporal Consistency
  * in KV-Cache Streaming" (t = absolute frame index).
@@ -144,6 +159,14 @@ LBM_API int lbm_cache_create(int heads, int head_dim, int patches_per_frame, int
 #define LBM_KEYFRAME_DEFERRED 2
 LBM_API int lbm_append_frame(lbm_cache_t* cache, void* q, const void* k, const void* v,
                      long long frame_idx, int is_keyframe, void* stream);
+/* The same for block block_idx of a multi-block cache.  Errors: LBM_ERR_INVALID for a block
+ * out of range or (blocks > 0) an is_keyframe different from block 0's; LBM_ERR_SEQUENCE
+ * unless block_idx is the next block of the frame in flight (block 0: no frame in flight;
+ * later blocks: the previous block has attended) and, for blocks > 0, frame_idx is that
+ * frame's. */
+LBM_API int lbm_append_frame_block(lbm_cache_t* cache, int block_idx, void* q, const void* k,
+                                   const void* v, long long frame_idx, int is_keyframe,
+                                   void* stream);
 
 /* Attention of the pending frame's (already rotated) queries over what the cache retains:
  * scale pages -> window pages (oldest first) -> the frame's own page -> all special tokens
@@ -157,6 +180,9 @@ LBM_API int lbm_append_frame(lbm_cache_t* cache, void* q, const void* k, const v
  * CTAs.  Errors: LBM_ERR_SEQUENCE if no frame is pending or the pending frame has already
  * been attended. */
 LBM_API int lbm_attend_frame(lbm_cache_t* cache, const void* q, void* out, void* stream);
+/* The same for block block_idx (LBM_ERR_SEQUENCE unless it has just appended). */
+LBM_API int lbm_attend_frame_block(lbm_cache_t* cache, int block_idx, const void* q, void* out,
+                                   void* stream);
 
 /* Keep (keep != 0) or drop the pending frame appended with LBM_KEYFRAME_DEFERRED, after its
  * attention ([KVBenefits] "Dynamic Keyframe Selection": a kept frame triggers the deferred
@@ -227,6 +253,9 @@ LBM_API int lbm_cache_state(const lbm_cache_t* cache, lbm_cache_state_t* state);
  * Elements are the cache's dtype. */
 LBM_API int lbm_cache_read_kv(const lbm_cache_t* cache, int which, int index, int count,
                       void* host_out);
+/* The same for block block_idx (lbm_cache_read_kv reads block 0). */
+LBM_API int lbm_cache_read_kv_block(const lbm_cache_t* cache, int block_idx, int which,
+                                    int index, int count, void* host_out);
 
 /* Synchronises the device and reports a bounded wait that ran out in an earlier kernel
  * (LBM_ERR_TIMEOUT, after which the error word is cleared) or LBM_OK. */

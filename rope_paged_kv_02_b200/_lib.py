@@ -33,8 +33,9 @@ LBM_MAX_PAGES = 1024
 # every symbol include/lbm.h declares
 SYMBOLS = [
     "lbm_rope3d_tables", "lbm_rope3d_tables_fhw", "lbm_rope3d_expand", "lbm_rope_destroy",
-    "lbm_cache_create", "lbm_append_frame", "lbm_attend_frame", "lbm_attend_frame_noalloc",
-    "lbm_commit_frame", "lbm_cache_reset",
+    "lbm_cache_create", "lbm_cache_create_blocks", "lbm_append_frame", "lbm_append_frame_block",
+    "lbm_attend_frame", "lbm_attend_frame_block", "lbm_attend_frame_noalloc",
+    "lbm_commit_frame", "lbm_cache_reset", "lbm_cache_read_kv_block",
     "lbm_cache_state", "lbm_cache_read_kv", "lbm_cache_check", "lbm_cache_destroy",
     "lbm_status_string",
     "lbm_pager_create", "lbm_pager_append", "lbm_pager_visible", "lbm_pager_finish",
@@ -95,6 +96,11 @@ def load() -> ctypes.CDLL:
     lib.lbm_rope_destroy.argtypes = [c_void]
     lib.lbm_rope_destroy.restype = None
     lib.lbm_cache_create.argtypes = [c_int] * 8 + [c_void, ctypes.POINTER(c_void)]
+    lib.lbm_cache_create_blocks.argtypes = [c_int] * 9 + [c_void, ctypes.POINTER(c_void)]
+    lib.lbm_append_frame_block.argtypes = [c_void, c_int, c_void, c_void, c_void, c_ll, c_int,
+                                           c_void]
+    lib.lbm_attend_frame_block.argtypes = [c_void, c_int, c_void, c_void, c_void]
+    lib.lbm_cache_read_kv_block.argtypes = [c_void, c_int, c_int, c_int, c_int, c_void]
     lib.lbm_append_frame.argtypes = [c_void, c_void, c_void, c_void, c_ll, c_int, c_void]
     lib.lbm_attend_frame.argtypes = [c_void, c_void, c_void, c_void]
     lib.lbm_attend_frame_noalloc.argtypes = [c_void, c_void, c_void, c_void]
@@ -217,16 +223,24 @@ class Rope3D:
 
 
 class PagedKVCache:
-    """lbm_cache_*: one layer's dual-stream paged KV cache on the current device."""
+    """lbm_cache_*: the dual-stream paged KV cache of one layer, or of num_blocks layers
+    sharing one page table, on the current device."""
 
     def __init__(self, rope: Rope3D, heads: int, head_dim: int, patches_per_frame: int,
                  scale_frames: int, sliding_window: int, max_frames: int, dtype: int,
-                 specials_per_frame: int = 6):
+                 specials_per_frame: int = 6, num_blocks: int = 1):
         lib = load()
         h = ctypes.c_void_p()
-        _check(lib.lbm_cache_create(heads, head_dim, patches_per_frame, specials_per_frame,
-                                    scale_frames, sliding_window, max_frames, dtype,
-                                    rope.handle, ctypes.byref(h)), "lbm_cache_create")
+        if num_blocks == 1:
+            _check(lib.lbm_cache_create(heads, head_dim, patches_per_frame, specials_per_frame,
+                                        scale_frames, sliding_window, max_frames, dtype,
+                                        rope.handle, ctypes.byref(h)), "lbm_cache_create")
+        else:
+            _check(lib.lbm_cache_create_blocks(num_blocks, heads, head_dim, patches_per_frame,
+                                               specials_per_frame, scale_frames, sliding_window,
+                                               max_frames, dtype, rope.handle, ctypes.byref(h)),
+                   "lbm_cache_create_blocks")
+        self.num_blocks = num_blocks
         self.handle = h
         self.rope = rope                      # the tables must outlive the cache
         self.heads, self.head_dim = heads, head_dim
@@ -244,6 +258,16 @@ class PagedKVCache:
                                        _keyframe_mode(is_keyframe), _stream(stream)),
                "lbm_append_frame")
 
+    def append_frame_block(self, block: int, q, k, v, frame_idx: int, is_keyframe,
+                           stream=None) -> None:
+        _check(load().lbm_append_frame_block(self.handle, int(block), _ptr(q), _ptr(k), _ptr(v),
+                                             int(frame_idx), _keyframe_mode(is_keyframe),
+                                             _stream(stream)), "lbm_append_frame_block")
+
+    def attend_frame_block(self, block: int, q, out, stream=None) -> None:
+        _check(load().lbm_attend_frame_block(self.handle, int(block), _ptr(q), _ptr(out),
+                                             _stream(stream)), "lbm_attend_frame_block")
+
     def commit_frame(self, keep: bool) -> None:
         _check(load().lbm_commit_frame(self.handle, 1 if keep else 0), "lbm_commit_frame")
 
@@ -258,13 +282,14 @@ class PagedKVCache:
         return _state_dict(lambda p: load().lbm_cache_state(self.handle, p),
                            max(self.num_pages, 1))
 
-    def read_kv(self, which: int, index: int, count: int = 0) -> np.ndarray:
+    def read_kv(self, which: int, index: int, count: int = 0, block: int = 0) -> np.ndarray:
         """Pool contents on the host: [heads, patches or count, head_dim], raw dtype."""
         rows = self.patches if which in (LBM_K_PATCH, LBM_V_PATCH) else count
         dt = np.uint16 if self.dtype == LBM_BF16 else np.float32
         out = np.empty((self.heads, rows, self.head_dim), dtype=dt)
-        _check(load().lbm_cache_read_kv(self.handle, which, index, count,
-                                        out.ctypes.data_as(ctypes.c_void_p)), "lbm_cache_read_kv")
+        _check(load().lbm_cache_read_kv_block(self.handle, int(block), which, index, count,
+                                              out.ctypes.data_as(ctypes.c_void_p)),
+               "lbm_cache_read_kv_block")
         return out
 
     def check(self) -> None:

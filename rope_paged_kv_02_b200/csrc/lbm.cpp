@@ -23,13 +23,22 @@ struct lbm_rope {
   int device = 0;
 };
 
+// K/V pools of one transformer block and their tensor maps.
+struct CacheBlock {
+  lbm::Pools pools{};
+  CUtensorMap tm_kp, tm_vp, tm_ks, tm_vs;
+};
+
 struct lbm_cache {
   int heads, head_dim, patches, psi, scale_frames, sliding_window, max_frames, dtype;
   int device = 0;
   int num_sms = 148;
   const lbm_rope* rope = nullptr;
-  lbm::Pools pools{};
-  void* pool_mem = nullptr;     // one allocation holding the four pools
+  std::vector<CacheBlock> blocks;  // one per transformer block, sharing the page table
+  int next_block = 0;           // block whose append / attention comes next in this frame
+  bool block_appended = false;  // next_block has appended this frame and not yet attended
+  int frame_mode = 0;           // is_keyframe of the frame in flight (0, 1, deferred)
+  void* pool_mem = nullptr;     // one allocation holding every block's four pools
   float* part_o = nullptr;      // partial outputs of units shared by several CTAs
   float* part_lse = nullptr;
   size_t scratch_floats = 0;    // capacity of part_o + part_lse in floats
@@ -37,7 +46,6 @@ struct lbm_cache {
   int* d_err = nullptr;
   long long device_bytes = 0;
   long long launches = 0;       // kernels launched so far
-  CUtensorMap tm_kp, tm_vp, tm_ks, tm_vs;
   CUtensorMap tm_q;             // cached for the last q pointer seen
   const void* tm_q_ptr = nullptr;
   lbm::Pager pager;
@@ -105,7 +113,8 @@ void order_after(lbm_cache* c, cudaStream_t s) {
 // Fills everything of the attention parameters but the partial-result scratch: the visible
 // page list (no container), tensor maps, and the stream-K partition of the frame's work
 // over the persistent CTAs.  Returns LBM_OK or an error status.
-int fill_attn_params(lbm_cache* c, const void* q, void* out, lbm::AttnParams& p) {
+int fill_attn_params(lbm_cache* c, int block, const void* q, void* out, lbm::AttnParams& p) {
+  const CacheBlock& bk = c->blocks[block];
   int n_pages = 0;
   for (const auto& e : c->pager.scale()) p.pages[n_pages++] = (uint16_t)e.page;
   for (const auto& e : c->pager.window()) p.pages[n_pages++] = (uint16_t)e.page;
@@ -119,16 +128,16 @@ int fill_attn_params(lbm_cache* c, const void* q, void* out, lbm::AttnParams& p)
     c->tm_q_ptr = q;
   }
   p.tm_q = c->tm_q;
-  p.tm_kp = c->tm_kp;
-  p.tm_vp = c->tm_vp;
-  p.tm_ks = c->tm_ks;
-  p.tm_vs = c->tm_vs;
+  p.tm_kp = bk.tm_kp;
+  p.tm_vp = bk.tm_vp;
+  p.tm_ks = bk.tm_ks;
+  p.tm_vs = bk.tm_vs;
   p.out = out;
   p.err = c->d_err;
   p.tokens = T;
   p.heads = c->heads;
   p.patches = c->patches;
-  p.page_stride = c->pools.page_stride;
+  p.page_stride = bk.pools.page_stride;
   p.tiles_per_page = (c->patches + kKeyTile - 1) / kKeyTile;
   p.n_pages = n_pages;
   p.n_special = n_sp;
@@ -141,6 +150,17 @@ int fill_attn_params(lbm_cache* c, const void* q, void* out, lbm::AttnParams& p)
   lbm::sk_partition(p);
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)c->head_dim));
   return LBM_OK;
+}
+
+// The attention of block next_block has been issued: the next block's turn, and after the
+// last block the frame is committed or rolled back (or, decided later, marked attended).
+void block_attended(lbm_cache* c) {
+  c->block_appended = false;
+  if (++c->next_block == (int)c->blocks.size()) {
+    c->next_block = 0;
+    int evicted = -1;
+    c->pager.finish(&evicted);
+  }
 }
 
 }  // namespace
@@ -247,8 +267,17 @@ void lbm_rope_destroy(lbm_rope_t* rope) {
 int lbm_cache_create(int heads, int head_dim, int patches_per_frame, int specials_per_frame,
                      int scale_frames, int sliding_window, int max_frames, int dtype,
                      const lbm_rope_t* rope, lbm_cache_t** out) {
+  return lbm_cache_create_blocks(1, heads, head_dim, patches_per_frame, specials_per_frame,
+                                 scale_frames, sliding_window, max_frames, dtype, rope, out);
+}
+
+int lbm_cache_create_blocks(int num_blocks, int heads, int head_dim, int patches_per_frame,
+                            int specials_per_frame, int scale_frames, int sliding_window,
+                            int max_frames, int dtype, const lbm_rope_t* rope,
+                            lbm_cache_t** out) {
   if (!out) return LBM_ERR_INVALID;
   *out = nullptr;
+  if (num_blocks < 1 || num_blocks > 1024) return LBM_ERR_INVALID;
   if (!rope || heads < 1 || heads > 65535 || patches_per_frame < 1 || scale_frames < 0 ||
       sliding_window < 0 || max_frames < 1 ||
       scale_frames + sliding_window + 1 > LBM_MAX_PAGES)
@@ -283,7 +312,8 @@ int lbm_cache_create(int heads, int head_dim, int patches_per_frame, int special
   const int e = elem_size(dtype);
   const size_t patch_bytes = (size_t)heads * P * stride * head_dim * e;
   const size_t spec_bytes = (size_t)heads * cap * head_dim * e;
-  const size_t total = 2 * patch_bytes + 2 * spec_bytes;
+  const size_t per_block = 2 * patch_bytes + 2 * spec_bytes;
+  const size_t total = per_block * (size_t)num_blocks;
   const int T = specials_per_frame + patches_per_frame;
   // partial results: (units + persistent CTAs) slots of 256 rows x (head_dim + 1) floats
   const long long units = (long long)(((T + 127) / 128 + 1) / 2) * heads;
@@ -313,25 +343,32 @@ int lbm_cache_create(int heads, int head_dim, int patches_per_frame, int special
   if (cudaMemset(c->d_err, 0, sizeof(int)) != cudaSuccess) return fail(LBM_ERR_CUDA);
   if (cudaEventCreateWithFlags(&c->ev, cudaEventDisableTiming) != cudaSuccess)
     return fail(LBM_ERR_CUDA);
-  char* base = static_cast<char*>(c->pool_mem);
-  c->pools.k_patch = base;
-  c->pools.v_patch = base + patch_bytes;
-  c->pools.k_special = base + 2 * patch_bytes;
-  c->pools.v_special = base + 2 * patch_bytes + spec_bytes;
-  c->pools.num_pages = P;
-  c->pools.page_stride = stride;
-  c->pools.spec_cap = (int)cap;
+  c->blocks.resize(num_blocks);
+  for (int b = 0; b < num_blocks; ++b) {
+    char* base = static_cast<char*>(c->pool_mem) + per_block * (size_t)b;
+    lbm::Pools& pl = c->blocks[b].pools;
+    pl.k_patch = base;
+    pl.v_patch = base + patch_bytes;
+    pl.k_special = base + 2 * patch_bytes;
+    pl.v_special = base + 2 * patch_bytes + spec_bytes;
+    pl.num_pages = P;
+    pl.page_stride = stride;
+    pl.spec_cap = (int)cap;
+  }
   c->device_bytes = (long long)(total + (dtype == LBM_BF16 ? part_o_bytes + part_lse_bytes : 0) +
                                 sizeof(int));
   if (dtype == LBM_BF16) {
     const uint64_t row = (uint64_t)head_dim * 2;
     const uint64_t prow = (uint64_t)P * stride;
     const uint32_t kt = kKeyTile;
-    if (!make_map(&c->tm_kp, c->pools.k_patch, head_dim, prow, heads, row, prow * row, kt, 1) ||
-        !make_map(&c->tm_vp, c->pools.v_patch, head_dim, prow, heads, row, prow * row, kt, 1) ||
-        !make_map(&c->tm_ks, c->pools.k_special, head_dim, cap, heads, row, cap * row, kt, 1) ||
-        !make_map(&c->tm_vs, c->pools.v_special, head_dim, cap, heads, row, cap * row, kt, 1))
-      return fail(LBM_ERR_CUDA);
+    for (CacheBlock& bk : c->blocks) {
+      const lbm::Pools& pl = bk.pools;
+      if (!make_map(&bk.tm_kp, pl.k_patch, head_dim, prow, heads, row, prow * row, kt, 1) ||
+          !make_map(&bk.tm_vp, pl.v_patch, head_dim, prow, heads, row, prow * row, kt, 1) ||
+          !make_map(&bk.tm_ks, pl.k_special, head_dim, cap, heads, row, cap * row, kt, 1) ||
+          !make_map(&bk.tm_vs, pl.v_special, head_dim, cap, heads, row, cap * row, kt, 1))
+        return fail(LBM_ERR_CUDA);
+    }
   }
   if (cudaDeviceSynchronize() != cudaSuccess) return fail(LBM_ERR_CUDA);
   *out = c;
@@ -340,15 +377,32 @@ int lbm_cache_create(int heads, int head_dim, int patches_per_frame, int special
 
 int lbm_append_frame(lbm_cache_t* c, void* q, const void* k, const void* v, long long frame_idx,
                      int is_keyframe, void* stream) {
+  if (!c) return LBM_ERR_INVALID;
+  return lbm_append_frame_block(c, c->next_block, q, k, v, frame_idx, is_keyframe, stream);
+}
+
+int lbm_append_frame_block(lbm_cache_t* c, int block, void* q, const void* k, const void* v,
+                           long long frame_idx, int is_keyframe, void* stream) {
   if (!c || !q || !k || !v || !aligned16(q) || !aligned16(k) || !aligned16(v))
     return LBM_ERR_INVALID;
   if (is_keyframe < 0 || is_keyframe > LBM_KEYFRAME_DEFERRED) return LBM_ERR_INVALID;
+  if (block < 0 || block >= (int)c->blocks.size()) return LBM_ERR_INVALID;
+  if (block != c->next_block || c->block_appended) return LBM_ERR_SEQUENCE;
   if (frame_idx < 0 || frame_idx >= c->rope->t.ppf) return LBM_ERR_SEQUENCE;
   int page = -1, slot = -1;
-  switch (c->pager.peek_append(frame_idx, is_keyframe, &page, &slot)) {
-    case lbm::PagerStatus::kOk: break;
-    case lbm::PagerStatus::kSequence: return LBM_ERR_SEQUENCE;
-    case lbm::PagerStatus::kCapacity: return LBM_ERR_CAPACITY;
+  if (block == 0) {
+    switch (c->pager.peek_append(frame_idx, is_keyframe, &page, &slot)) {
+      case lbm::PagerStatus::kOk: break;
+      case lbm::PagerStatus::kSequence: return LBM_ERR_SEQUENCE;
+      case lbm::PagerStatus::kCapacity: return LBM_ERR_CAPACITY;
+    }
+  } else {
+    // a later block writes the same frame into its own pools, at the page and special
+    // slots block 0 took
+    if (!c->pager.pending() || frame_idx != c->pager.pending_frame()) return LBM_ERR_SEQUENCE;
+    if (is_keyframe != c->frame_mode) return LBM_ERR_INVALID;
+    page = c->pager.pending_page();
+    slot = c->pager.n_special();
   }
   if (use_device(c->device) != LBM_OK) return LBM_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -365,10 +419,15 @@ int lbm_append_frame(lbm_cache_t* c, void* q, const void* k, const void* v, long
   a.k = k;
   a.v = v;
   order_before(c, s);
-  if (lbm::launch_rope_append(c->rope->t, c->pools, a, s) != cudaSuccess) return LBM_ERR_CUDA;
+  if (lbm::launch_rope_append(c->rope->t, c->blocks[block].pools, a, s) != cudaSuccess)
+    return LBM_ERR_CUDA;
   ++c->launches;
   order_after(c, s);
-  c->pager.append(frame_idx, is_keyframe, &page, &slot);
+  if (block == 0) {
+    c->pager.append(frame_idx, is_keyframe, &page, &slot);
+    c->frame_mode = is_keyframe;
+  }
+  c->block_appended = true;
   return LBM_OK;
 }
 
@@ -384,19 +443,26 @@ int lbm_commit_frame(lbm_cache_t* c, int keep) {
 }
 
 int lbm_attend_frame(lbm_cache_t* c, const void* q, void* out, void* stream) {
+  if (!c) return LBM_ERR_INVALID;
+  return lbm_attend_frame_block(c, c->next_block, q, out, stream);
+}
+
+int lbm_attend_frame_block(lbm_cache_t* c, int block, const void* q, void* out, void* stream) {
   if (!c || !q || !out || !aligned16(q) || !aligned16(out)) return LBM_ERR_INVALID;
+  if (block < 0 || block >= (int)c->blocks.size()) return LBM_ERR_INVALID;
   std::vector<int> pages;
   int n_sp = 0, last_len = 0;
-  if (!c->pager.awaiting_attention() ||
+  if (block != c->next_block || !c->block_appended || !c->pager.awaiting_attention() ||
       c->pager.visible(&pages, &n_sp, &last_len) != lbm::PagerStatus::kOk)
     return LBM_ERR_SEQUENCE;
+  const lbm::Pools& pl = c->blocks[block].pools;
   if (use_device(c->device) != LBM_OK) return LBM_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int T = c->psi + c->patches;
   order_before(c, s);
   if (c->dtype == LBM_BF16) {
-    static thread_local lbm::AttnParams p;  // ~3 KB: kept off the stack
-    const int st = fill_attn_params(c, q, out, p);
+    static thread_local lbm::AttnParams p;  // ~7 KB: kept off the stack
+    const int st = fill_attn_params(c, block, q, out, p);
     if (st != LBM_OK) return st;
     const long long units = (long long)p.n_pairs * c->heads;
     if (lbm::sk_scratch_floats(units, p.grid, c->head_dim) > c->scratch_floats)
@@ -413,17 +479,17 @@ int lbm_attend_frame(lbm_cache_t* c, const void* q, void* out, void* stream) {
     static thread_local lbm::SimtParams p;
     p.q = q;
     p.out = out;
-    p.k_patch = c->pools.k_patch;
-    p.v_patch = c->pools.v_patch;
-    p.k_special = c->pools.k_special;
-    p.v_special = c->pools.v_special;
+    p.k_patch = pl.k_patch;
+    p.v_patch = pl.v_patch;
+    p.k_special = pl.k_special;
+    p.v_special = pl.v_special;
     p.tokens = T;
     p.heads = c->heads;
     p.head_dim = c->head_dim;
     p.patches = c->patches;
-    p.page_stride = c->pools.page_stride;
-    p.pool_pages = c->pools.num_pages;
-    p.spec_cap = c->pools.spec_cap;
+    p.page_stride = pl.page_stride;
+    p.pool_pages = pl.num_pages;
+    p.spec_cap = pl.spec_cap;
     p.n_pages = (int)pages.size();
     p.n_special = n_sp;
     p.scale = (float)(1.0 / std::sqrt((double)c->head_dim));
@@ -432,22 +498,22 @@ int lbm_attend_frame(lbm_cache_t* c, const void* q, void* out, void* stream) {
     ++c->launches;
   }
   order_after(c, s);
-  int evicted = -1;
-  c->pager.finish(&evicted);
+  block_attended(c);
   return LBM_OK;
 }
 
 int lbm_attend_frame_noalloc(lbm_cache_t* c, const void* q, void* out, void* stream) {
   if (!c || !q || !out || !aligned16(q) || !aligned16(out)) return LBM_ERR_INVALID;
   if (c->dtype != LBM_BF16) return LBM_ERR_UNSUPPORTED;
-  if (!c->pager.awaiting_attention()) return LBM_ERR_SEQUENCE;
+  if (!c->block_appended || !c->pager.awaiting_attention()) return LBM_ERR_SEQUENCE;
+  const int block = c->next_block;
   if (use_device(c->device) != LBM_OK) return LBM_ERR_CUDA;
   float* scratch = nullptr;
   size_t scratch_floats = 0;
   const int st = lbm::noalloc_scratch(c->device, &scratch, &scratch_floats);
   if (st != LBM_OK) return st;
   lbm::AttnParams p;  // on the stack: this call touches no heap
-  const int pst = fill_attn_params(c, q, out, p);
+  const int pst = fill_attn_params(c, block, q, out, p);
   if (pst != LBM_OK) return pst;
   const long long units = (long long)p.n_pairs * c->heads;
   const bool split = lbm::sk_has_split(p);
@@ -464,14 +530,15 @@ int lbm_attend_frame_noalloc(lbm_cache_t* c, const void* q, void* out, void* str
     ++c->launches;
   }
   order_after(c, s);
-  int evicted = -1;
-  c->pager.finish(&evicted);
+  block_attended(c);
   return LBM_OK;
 }
 
 int lbm_cache_reset(lbm_cache_t* c) {
   if (!c) return LBM_ERR_INVALID;
   c->pager.reset();
+  c->next_block = 0;
+  c->block_appended = false;
   return LBM_OK;
 }
 
@@ -483,24 +550,30 @@ int lbm_cache_state(const lbm_cache_t* c, lbm_cache_state_t* st) {
 }
 
 int lbm_cache_read_kv(const lbm_cache_t* c, int which, int index, int count, void* host_out) {
-  if (!c || !host_out) return LBM_ERR_INVALID;
+  return lbm_cache_read_kv_block(c, 0, which, index, count, host_out);
+}
+
+int lbm_cache_read_kv_block(const lbm_cache_t* c, int block, int which, int index, int count,
+                            void* host_out) {
+  if (!c || !host_out || block < 0 || block >= (int)c->blocks.size()) return LBM_ERR_INVALID;
+  const lbm::Pools& pl = c->blocks[block].pools;
   const int e = elem_size(c->dtype);
   const size_t row = (size_t)c->head_dim * e;
   const void* src;
   size_t pitch, width;
   if (which == LBM_K_PATCH || which == LBM_V_PATCH) {
-    if (index < 0 || index >= c->pools.num_pages) return LBM_ERR_INVALID;
-    const char* pool = static_cast<const char*>(which == LBM_K_PATCH ? c->pools.k_patch
-                                                                     : c->pools.v_patch);
-    src = pool + (size_t)index * c->pools.page_stride * row;
-    pitch = (size_t)c->pools.num_pages * c->pools.page_stride * row;
+    if (index < 0 || index >= pl.num_pages) return LBM_ERR_INVALID;
+    const char* pool = static_cast<const char*>(which == LBM_K_PATCH ? pl.k_patch
+                                                                     : pl.v_patch);
+    src = pool + (size_t)index * pl.page_stride * row;
+    pitch = (size_t)pl.num_pages * pl.page_stride * row;
     width = (size_t)c->patches * row;
   } else if (which == LBM_K_SPECIAL || which == LBM_V_SPECIAL) {
-    if (index < 0 || count < 1 || index + count > c->pools.spec_cap) return LBM_ERR_INVALID;
-    const char* pool = static_cast<const char*>(which == LBM_K_SPECIAL ? c->pools.k_special
-                                                                       : c->pools.v_special);
+    if (index < 0 || count < 1 || index + count > pl.spec_cap) return LBM_ERR_INVALID;
+    const char* pool = static_cast<const char*>(which == LBM_K_SPECIAL ? pl.k_special
+                                                                       : pl.v_special);
     src = pool + (size_t)index * row;
-    pitch = (size_t)c->pools.spec_cap * row;
+    pitch = (size_t)pl.spec_cap * row;
     width = (size_t)count * row;
   } else {
     return LBM_ERR_INVALID;

@@ -257,3 +257,79 @@ def test_calls_on_two_streams_are_ordered():
         check_attn(host(out), r.out, f"frame {f}")
     cache.close()
     rope.close()
+
+
+def test_multi_block_cache_shares_the_page_table():
+    """[3DRoPE-KV] "Implementation Example": one cache manager for several transformer blocks
+    (num_blocks, block_idx).  Three blocks with their own seeded inputs stream the same frames
+    (append then attend per block, blocks in order); each block's outputs and pages match its
+    own oracle, and the shared page table matches every oracle's."""
+    import torch
+    from oracle import stream as ostream
+    from stream_check import check_attn, check_rope, dev, host, pool_values
+    from rope_paged_kv_02_b200 import workloads
+    nb = 3
+    cfgs = [custom_config(215 + b, 2, 64, "bf16", 5, 6, 9, 2, 1, 2) for b in range(nb)]
+    c0 = cfgs[0]
+    rope = _lib.Rope3D(64, c0.n_frames, c0.pph, c0.ppw, 6)
+    cache = _lib.PagedKVCache(rope, 2, 64, c0.patches, c0.scale_frames, c0.sliding_window,
+                              c0.n_keyframes, _lib.LBM_BF16, num_blocks=nb)
+    oracles = [ostream.StreamOracle(2, 64, c0.pph, c0.ppw, c0.scale_frames, c0.sliding_window,
+                                    c0.n_keyframes) for _ in range(nb)]
+    for f in range(c0.n_frames):
+        key = c0.keyframes[f]
+        for b in range(nb):
+            q, k, v = workloads.frame_qkv(cfgs[b], f)
+            qd, kd, vd = dev(q, "bf16"), dev(k, "bf16"), dev(v, "bf16")
+            out = torch.empty_like(qd)
+            cache.append_frame_block(b, qd, kd, vd, f, key)
+            cache.attend_frame_block(b, qd, out)
+            r = oracles[b].step(f, key, q, k, v)
+            torch.cuda.synchronize()
+            check_rope(host(qd), r.q_rot, "bf16", f"block {b} frame {f} q")
+            check_attn(host(out), r.out, f"block {b} frame {f} attention")
+            kp = pool_values(cache.read_kv(_lib.LBM_K_PATCH, r.page, block=b), "bf16")
+            check_rope(kp.transpose(1, 0, 2), r.k_rot[6:], "bf16", f"block {b} K page")
+            vp = pool_values(cache.read_kv(_lib.LBM_V_PATCH, r.page, block=b), "bf16")
+            np.testing.assert_array_equal(vp.transpose(1, 0, 2), v[6:])
+            st = cache.state()
+            assert st["pending"] == (b < nb - 1)       # committed after the last block
+        for b in range(nb):
+            snap = oracles[b].ret.snapshot()
+            for k_ in ("scale_pages", "scale_frames", "window_pages", "window_frames", "free",
+                       "n_special"):
+                assert st[k_] == snap[k_], (f, b, k_)
+    cache.check()
+    cache.close()
+    rope.close()
+
+
+def test_multi_block_sequence_errors():
+    import torch
+    rope = _lib.Rope3D(64, 4, 4, 4, 6)
+    cache = _lib.PagedKVCache(rope, 2, 64, 16, 1, 1, 4, _lib.LBM_BF16, num_blocks=2)
+    q = torch.randn(22, 2, 64, device="cuda").to(torch.bfloat16)
+    k, v, out = torch.randn_like(q), torch.randn_like(q), torch.empty_like(q)
+
+    def status(fn, *a):
+        with pytest.raises(_lib.LbmError) as e:
+            fn(*a)
+        return e.value.status
+
+    assert status(cache.append_frame_block, 1, q, k, v, 0, True) == _lib.LBM_ERR_SEQUENCE
+    assert status(cache.append_frame_block, 2, q, k, v, 0, True) == _lib.LBM_ERR_INVALID
+    cache.append_frame_block(0, q, k, v, 0, True)
+    assert status(cache.append_frame_block, 1, q, k, v, 0, True) == _lib.LBM_ERR_SEQUENCE
+    assert status(cache.attend_frame_block, 1, q, out) == _lib.LBM_ERR_SEQUENCE
+    cache.attend_frame_block(0, q, out)
+    assert status(cache.attend_frame_block, 0, q, out) == _lib.LBM_ERR_SEQUENCE
+    assert status(cache.append_frame_block, 1, q, k, v, 1, True) == _lib.LBM_ERR_SEQUENCE
+    assert status(cache.append_frame_block, 1, q, k, v, 0, False) == _lib.LBM_ERR_INVALID
+    s0 = cache.state()
+    assert s0["pending"]
+    cache.append_frame(q, k, v, 0, True)                  # the next block in order: block 1
+    cache.attend_frame(q, out)
+    assert not cache.state()["pending"] and cache.state()["scale_frames"] == [0]
+    cache.check()
+    cache.close()
+    rope.close()
