@@ -172,6 +172,23 @@ def test_long_stream_2000_keyframes_sampled():
                check_pools=False)
 
 
+@pytest.mark.parametrize("head_dim", [64, 128])
+def test_single_patch_frames(head_dim):
+    """The smallest frame: 6 special tokens and one patch (T = 7, one mostly padded query
+    tile, one-key patch pages)."""
+    run_stream(custom_config(218 + head_dim // 64, 1, head_dim, "bf16", 1, 1, 9, 2, 1, 2))
+
+
+@pytest.mark.slow
+def test_maximum_page_count():
+    """The largest page table the cache takes (scale_frames + sliding_window + 1 = 1024 =
+    LBM_MAX_PAGES) over a stream long enough to fill and roll it: the kernel's visible page
+    list is full, and each unit's ~1000 key tiles are spread over every CTA, so the combine
+    merges ~70 partials a row."""
+    cfg = custom_config(221, 2, 64, "bf16", 4, 4, 1030, 1, 8, 1015)
+    run_stream(cfg, check_frames=[0, 1, 1022, 1023, 1024, 1029], regenerate=True)
+
+
 def test_sequence_errors_leave_state_unchanged():
     import torch
     cfg = custom_config(208, 2, 64, "bf16", 4, 4, 4, 1, 1, 1)
