@@ -3,9 +3,9 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config C]
 
 One step streams every frame of the workload through a fresh cache: per frame one
-lbm_append_frame (fused rotate + append) and one lbm_attend_frame (paged attention, plus
-the split-KV combine when the planner splits the keys), host page-table bookkeeping
-included.  The default workload is the 768-patch stream: 16 heads x head_dim 64, bf16,
+lbm_append_frame (fused rotate + append) and one lbm_attend_frame (paged attention on
+persistent CTAs, plus the combine of the units several CTAs share), host page-table
+bookkeeping included.  The default workload is the 768-patch stream: 16 heads x head_dim 64, bf16,
 6 special + 24x32 patch tokens per frame, 64 keyframes, scale_frames 8, sliding_window 16.
 Inputs are seeded synthetic frames; the 64 frames of a step (304 MB of q/k/v) are larger
 than L2, so no input is L2-resident between steps.

@@ -23,7 +23,7 @@
  *  - stream is a cudaStream_t (NULL = the legacy default stream).  Work is only enqueued;
  *    nothing synchronises the host except the calls that say so.  Calls on one cache from
  *    several streams are ordered by the library through an event it records after each launch.
- *  - The library owns the RoPE tables, the K/V page pools, split-KV scratch and the page
+ *  - The library owns the RoPE tables, the K/V page pools, stream-K scratch and the page
  *    table.  The caller owns its q/k/v/out buffers and the streams.
  *  - Host bookkeeping (page table, free list, deferred eviction) runs at call time on the
  *    host; the only host->device traffic of a frame is kernel launch parameters.
@@ -121,7 +121,8 @@ LBM_API void lbm_rope_destroy(lbm_rope_t* rope);
  * Device memory: K and V patch pools [heads][P*stride][head_dim] with P = scale_frames +
  * sliding_window + 1 pages and stride = patches_per_frame rounded up to 128 (zero-filled);
  * K and V special pools [heads][cap][head_dim], cap = 6*(max_frames+1) rounded up to 128;
- * split-KV scratch.  Synchronous. */
+ * stream-K scratch: partial results of (units + persistent CTAs) x 256 rows x (head_dim + 1)
+ * floats, a unit being one (pair of 128-row query tiles, head).  Synchronous. */
 LBM_API int lbm_cache_create(int heads, int head_dim, int patches_per_frame, int specials_per_frame,
                      int scale_frames, int sliding_window, int max_frames, int dtype,
                      const lbm_rope_t* rope, lbm_cache_t** out);
@@ -196,15 +197,15 @@ LBM_API int lbm_commit_frame(lbm_cache_t* cache, int keep);
  * stream (a runtime that owns the whole GPU through its own pool and budget, or a real-time
  * loop where cudaMalloc / cudaFree would synchronise the device).  The pages describe no such
  * call; it has no counterpart there.  Same arguments, same result and same page-table update
- * as lbm_attend_frame, but the split-KV partial results go to a file-scope device array of
+ * as lbm_attend_frame, but the stream-K partial results go to a file-scope device array of
  * LBM_NOALLOC_SCRATCH_BYTES (16 MiB) that every GPU loading the library holds until exit,
  * instead of the cache's own scratch; the call allocates nothing (device or host heap).
  *   - bf16 caches only (LBM_ERR_UNSUPPORTED otherwise).
  *   - The first call on a device looks up the array's device address with that device
  *     current; make that first call before any stream capture.
- *   - A frame whose planned key split needs more than LBM_NOALLOC_SCRATCH_BYTES of partial
- *     results (splits x T x heads x (head_dim + 1) x 4 bytes) is refused with
- *     LBM_ERR_CAPACITY and the cache is left as it was.
+ *   - A frame whose units are shared by CTAs and whose partial results need more than
+ *     LBM_NOALLOC_SCRATCH_BYTES ((units + CTAs) x 256 x (head_dim + 1) x 4 bytes) is refused
+ *     with LBM_ERR_CAPACITY and the cache is left as it was.
  *   - Every call shares the array and leaves its last contents there; nothing in it needs
  *     to start at zero.  Calls whose kernels overlap on the GPU (several streams or caches
  *     at once) race on it: order them. */

@@ -1,9 +1,9 @@
-// Split-KV scratch that lives in a file-scope device array, for lbm_attend_frame_noalloc.
+// Stream-K scratch that lives in a file-scope device array, for lbm_attend_frame_noalloc.
 //
 // Some callers of this library may not allocate device memory while frames stream: a
 // serving runtime that owns every byte of the GPU through its own pool and budget, or a
 // real-time frame loop where cudaMalloc / cudaFree would synchronise the device and stall
-// the stream.  lbm_attend_frame_noalloc serves them: its split-KV partial results go to the
+// the stream.  lbm_attend_frame_noalloc serves them: its stream-K partial results go to the
 // array below, which the CUDA runtime places when the library is loaded, so the call itself
 // allocates nothing.
 //

@@ -163,7 +163,7 @@ inline bool sk_has_split(const AttnParams& p) {
   return false;
 }
 
-// attn_static.cu: device address of the file-scope split-KV scratch on `device` (current)
+// attn_static.cu: device address of the file-scope stream-K scratch on `device` (current)
 int noalloc_scratch(int device, float** ptr, size_t* floats);
 
 // attn_simt.cu (fp32)

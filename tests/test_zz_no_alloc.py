@@ -3,7 +3,7 @@
 The no-allocation entry point exists for callers that may not allocate device memory while
 frames stream (a runtime that owns the GPU through its own pool, a real-time loop where
 cudaMalloc would synchronise the device).  It must give the same attention output and the
-same page-table update as the regular call while taking its split-KV scratch from the
+same page-table update as the regular call while taking its stream-K scratch from the
 library's file-scope device array.  Two caches receive the identical seeded stream; frame
 by frame, one is attended with each entry point (several calls in a row), and the outputs
 are compared with the tolerance the parity tests use.  This file is collected last on
