@@ -438,8 +438,11 @@ def main():
 
 def e2e_measure(cfg, cache, args, dev, tdt, world):
     """Same metric through the C ABI with host buffers: per frame, pinned host q/k/v are
-    copied to the device on a copy stream (overlapping the previous frame's kernels), the
-    frame is appended and attended, and its output is copied back to pinned host memory."""
+    copied to the device on a host-to-device stream, the frame is appended and attended on
+    the compute stream, and its output is copied back to pinned host memory on a
+    device-to-host stream, so both copies overlap other frames' kernels.  Three device
+    buffer sets rotate: a frame's inputs are overwritten only after the frame that last used
+    them has been attended, its output only after the previous one has been copied out."""
     import torch
     F = cfg.n_frames
     from rope_paged_kv_02_b200 import workloads
@@ -451,43 +454,53 @@ def e2e_measure(cfg, cache, args, dev, tdt, world):
         hk.append(torch.from_numpy(k).to(tdt).pin_memory())
         hv.append(torch.from_numpy(v).to(tdt).pin_memory())
         ho.append(torch.empty_like(hq[-1]).pin_memory())
-    nbuf = 2
+    nbuf = 3
     dq = [torch.empty(hq[0].shape, dtype=tdt, device=dev) for _ in range(nbuf)]
     dk = [torch.empty_like(dq[0]) for _ in range(nbuf)]
     dv = [torch.empty_like(dq[0]) for _ in range(nbuf)]
     do = [torch.empty_like(dq[0]) for _ in range(nbuf)]
     comp = torch.cuda.current_stream(dev)
-    copy = torch.cuda.Stream(dev)
-    done = [torch.cuda.Event() for _ in range(nbuf)]   # buffer free (its frame finished)
-    ready = [torch.cuda.Event() for _ in range(nbuf)]  # inputs landed
+    h2d = torch.cuda.Stream(dev)
+    d2h = torch.cuda.Stream(dev)
+    attended = [torch.cuda.Event() for _ in range(nbuf)]  # the frame in buffer b attended
+    landed = [torch.cuda.Event() for _ in range(nbuf)]    # inputs of buffer b on the device
+    copied = [torch.cuda.Event() for _ in range(nbuf)]    # output of buffer b on the host
     keys = cfg.keyframes
 
-    def step():
+    def step(first):
         cache.reset()
         for f in range(F):
             b = f % nbuf
             h = f % pool
-            with torch.cuda.stream(copy):
-                copy.wait_event(done[b])
+            reuse = not first or f >= nbuf
+            with torch.cuda.stream(h2d):
+                if reuse:
+                    h2d.wait_event(attended[b])
                 dq[b].copy_(hq[h], non_blocking=True)
                 dk[b].copy_(hk[h], non_blocking=True)
                 dv[b].copy_(hv[h], non_blocking=True)
-                ready[b].record(copy)
-            comp.wait_event(ready[b])
+                landed[b].record(h2d)
+            comp.wait_event(landed[b])
+            if reuse:
+                comp.wait_event(copied[b])
             cache.append_frame(dq[b], dk[b], dv[b], f, keys[f], comp)
             cache.attend_frame(dq[b], do[b], comp)
-            ho[f % pool].copy_(do[b], non_blocking=True)
-            done[b].record(comp)
+            attended[b].record(comp)
+            with torch.cuda.stream(d2h):
+                d2h.wait_event(attended[b])
+                ho[h].copy_(do[b], non_blocking=True)
+                copied[b].record(d2h)
 
-    for _ in range(2):
-        step()
+    step(True)
+    step(False)
     torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
     t0.record(comp)
     for _ in range(args.steps):
-        step()
+        step(False)
+    comp.wait_stream(d2h)          # the last outputs are on the host
     t1.record(comp)
     torch.cuda.synchronize()
     ms = max_over_ranks(t0.elapsed_time(t1), world)
