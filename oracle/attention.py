@@ -5,7 +5,7 @@ TEST INFRASTRUCTURE ONLY (see ``oracle/__init__``).
 [3DRoPE-KV] "Attention Computation with Cached RoPE": the frame's queries attend over the
 visible pages with K/V that already carry their rotation.  [RealTime3D] "Per-Frame
 Processing and Causal Attention": a frame sees cached past tokens and special tokens, no
-future frame.  Reading: a frame's own tokens are all visible to each other
+future frame.  Reading where the pages are loose: a frame's own tokens are all visible to each other
 (bidirectional inside the frame); scale is 1/sqrt(head_dim).
 
 Two formulations, which must agree:

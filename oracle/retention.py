@@ -16,7 +16,7 @@ What the pages fix
   non-keyframes are processed but not cached; a kept frame triggers the deferred eviction,
   a dropped frame's temporary entry is rolled back.
 
-Readings (listed in DESIGN.md):
+Readings where the pages leave a step open:
 
 * A frame is appended tentatively, attends (its own tokens visible), then is committed
   (keyframe) or rolled back (non-keyframe).  Eviction happens at commit, i.e. after the

@@ -20,7 +20,7 @@ What the pages fix
 * [VideoRoPE] "Temporal Consistency in KV-Cache Streaming": the t coordinate is the
   absolute (global) frame index of the stream.
 
-Readings where the pages leave a step open (each listed in the design doc):
+Readings where the pages leave a step open:
 
 * inv_freq of axis a with ``d_a`` features: ``theta ** (-(2 i) / d_a)``, ``i < d_a / 2``.
 * Split of ``head_dim``: ``d_h = d_w = 2 * (head_dim // 6)``, ``d_t = head_dim - 2 d_h``
