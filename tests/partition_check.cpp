@@ -1,0 +1,60 @@
+// Host check of the stream-K partition the attention launcher uses (sk_partition): for many
+// frame shapes and grid sizes, the CTA starts begin at 0, end at the frame's work, strictly
+// increase (every CTA gets work), and no CTA's modelled cost exceeds the even share by more
+// than one unit's start plus a step.  Built and run by tests/test_partition_host.py.
+#include <cstdio>
+#include <algorithm>
+#include "../rope_paged_kv_02_b200/csrc/lbm_internal.h"
+
+using namespace lbm;
+
+static AttnParams p;  // large: static storage
+
+int main() {
+  long long checked = 0;
+  for (int T : {7, 22, 128, 129, 256, 300, 774, 1005, 4102})
+    for (int H : {1, 2, 8, 16, 40})
+      for (int nt : {1, 2, 3, 7, 153, 1090})
+        for (int want : {1, 2, 3, 16, 100, 148, 592, 1024}) {
+          p.tokens = T;
+          p.heads = H;
+          p.n_tiles = nt;
+          p.n_pairs = ((T + 127) / 128 + 1) / 2;
+          p.work = (long long)p.n_pairs * H * nt;
+          p.grid = (int)std::min<long long>(std::min<long long>(want, p.work), kMaxGrid);
+          sk_partition(p);
+          if (p.sk_start[0] != 0 || p.sk_start[p.grid] != p.work) {
+            std::printf("FAIL ends T=%d H=%d nt=%d grid=%d\n", T, H, nt, p.grid);
+            return 1;
+          }
+          const bool single_last = ((T + 127) / 128) % 2 == 1;
+          long long total = 0, worst = 0;
+          for (int c = 0; c < p.grid; ++c) {
+            if (p.sk_start[c + 1] <= p.sk_start[c]) {
+              std::printf("FAIL empty share T=%d H=%d nt=%d grid=%d c=%d\n", T, H, nt, p.grid, c);
+              return 1;
+            }
+            long long cost = 0;
+            for (int x = p.sk_start[c]; x < p.sk_start[c + 1]; ++x) {
+              const int unit = x / nt;
+              const bool single = single_last && unit % p.n_pairs == p.n_pairs - 1;
+              if (x == p.sk_start[c] || x % nt == 0) cost += kCostSegment;
+              cost += single ? kCostSingleStep : kCostPairStep;
+            }
+            total += cost;
+            worst = std::max(worst, cost);
+          }
+          // the even share plus what one boundary can add: a segment start and a step, plus
+          // the steps the non-empty rule may move onto a CTA when shares are tiny
+          const long long even = (total + p.grid - 1) / p.grid;
+          const long long slack = kCostSegment + 2 * kCostPairStep;
+          if (p.work >= 4LL * p.grid && worst > even + slack) {
+            std::printf("FAIL balance T=%d H=%d nt=%d grid=%d worst=%lld even=%lld\n", T, H, nt,
+                        p.grid, worst, even);
+            return 1;
+          }
+          ++checked;
+        }
+  std::printf("ok %lld\n", checked);
+  return 0;
+}
