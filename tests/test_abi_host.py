@@ -200,3 +200,13 @@ def test_create_argument_checks_without_gpu(lib):
     assert lib.lbm_attend_frame(None, None, None, None) == _lib.LBM_ERR_INVALID
     assert lib.lbm_cache_reset(None) == _lib.LBM_ERR_INVALID
     assert lib.lbm_cache_check(None) == _lib.LBM_ERR_INVALID
+    assert lib.lbm_commit_frame(None, 1) == _lib.LBM_ERR_INVALID
+    # multi-block caches: block count checked first; block calls on a null cache
+    for nb in (0, -1, 1025):
+        assert lib.lbm_cache_create_blocks(nb, 2, 64, 16, 6, 1, 3, 8, _lib.LBM_BF16, None,
+                                           ctypes.byref(h)) == _lib.LBM_ERR_INVALID
+    assert lib.lbm_append_frame_block(None, 0, None, None, None, 0, 1,
+                                      None) == _lib.LBM_ERR_INVALID
+    assert lib.lbm_attend_frame_block(None, 0, None, None, None) == _lib.LBM_ERR_INVALID
+    buf = ctypes.create_string_buffer(16)
+    assert lib.lbm_cache_read_kv_block(None, 0, 0, 0, 0, buf) == _lib.LBM_ERR_INVALID
