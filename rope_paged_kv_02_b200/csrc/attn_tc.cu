@@ -13,16 +13,18 @@
 //               tcgen05.mma of query tile g:
 //                 S = Q_g K_j^T   (A, B from shared memory)      -> TMEM S_g
 //                 O_g += P V_j    (A = P from TMEM, B = V smem)   -> TMEM O_g
-//               With head_dim 64, S_{j+1} is issued as soon as the softmax warps have read
-//               S_j, before PV_j, so scores and softmax overlap.
+//               S_{j+1} is issued before PV_j, so scores and softmax overlap: at head_dim 64
+//               as soon as the softmax warps have read S_j (one S buffer); at head_dim 128
+//               into the other of two S buffers once PV_{j-1} has read the P it held.
 //   warps 4..7  softmax of query tile 0, warps 8..11 of tile 1: each thread owns one query
 //               row (its TMEM lane); reads S_j, row max, exp2, row sum in fp32, writes P_j
 //               (bf16) into TMEM, and rescales O only when the running max grew by more than
 //               2^8 (lazy rescale; exact because O and l share one reference max).
 //   The two softmax warpgroups run concurrently, so one's exponentials overlap the other's
 //   tensor-core work.
-// Tensor memory: 256 columns per query tile g at 256 g: S [0,128); head_dim 64:
-// P [128,192), O [192,256); head_dim 128: O [128,256), P written over S [0,64).
+// Tensor memory: 256 columns per query tile g at 256 g.  head_dim 64, 128-key tiles: S [0,128),
+// P [128,192), O [192,256).  head_dim 128, 64-key tiles: S_0 [0,64), S_1 [64,128) with P_b
+// written over S_b, O [128,256).
 // Every mbarrier wait is bounded (about 2 s); a wait that runs out sets the device error
 // word, raises a CTA-wide abort flag, and every role falls through to the common exit,
 // which drains outstanding copies / MMAs (bounded) and frees tensor memory.
@@ -35,7 +37,6 @@ namespace lbm {
 namespace {
 
 constexpr int BM = 128;         // query rows per CTA
-constexpr int BN = 128;         // keys per tile
 constexpr int kThreads = 384;   // 12 warps
 constexpr uint32_t kTmemCols = 512;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
@@ -46,15 +47,18 @@ constexpr int kMaxStages = 4;  // K/V ring stages the barrier block has room for
 
 template <int D>
 struct Cfg {
-  static constexpr int NS = D == 64 ? 4 : 2;            // K/V pipeline stages
+  static constexpr int BN = attn_key_tile(D);            // keys per K/V tile
+  static constexpr int NS = 4;                           // K/V pipeline stages
   static_assert(NS <= kMaxStages, "the barrier block holds kMaxStages ring barriers");
-  static constexpr int ATOM_BYTES = 128 * 128;          // 128 rows x 64 bf16 (one swizzle atom column)
-  static constexpr int ATOMS = D / 64;
-  static constexpr int TILE_BYTES = ATOMS * ATOM_BYTES; // one Q, K or V tile
-  static constexpr int OFF_Q = 0;                       // two query tiles
-  static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
-  static constexpr int OFF_V = OFF_K + NS * TILE_BYTES;
-  static constexpr int OFF_BAR = OFF_V + NS * TILE_BYTES;
+  static constexpr int ATOMS = D / 64;                   // 64-feature swizzle atom columns
+  static constexpr int Q_ATOM = BM * 128;                // 128 query rows x 64 bf16
+  static constexpr int KV_ATOM = BN * 128;               // BN key rows x 64 bf16
+  static constexpr int Q_TILE = ATOMS * Q_ATOM;          // one query tile
+  static constexpr int KV_TILE = ATOMS * KV_ATOM;        // one K or V tile
+  static constexpr int OFF_Q = 0;                        // two query tiles
+  static constexpr int OFF_K = OFF_Q + 2 * Q_TILE;
+  static constexpr int OFF_V = OFF_K + NS * KV_TILE;
+  static constexpr int OFF_BAR = OFF_V + NS * KV_TILE;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM = OFF_BAR + BAR_BYTES + 1024;  // + slack to align the base to 1 KB
 };
@@ -288,6 +292,7 @@ struct TileRef {
   int valid;
 };
 
+template <int BN>
 __device__ __forceinline__ TileRef tile_ref(const AttnParams& p, int t) {
   const int npt = p.n_pages * p.tiles_per_page;
   TileRef r;
@@ -309,10 +314,10 @@ __device__ __forceinline__ TileRef tile_ref(const AttnParams& p, int t) {
 struct Bars {
   uint64_t q_full;         // the query tiles of the current segment landed
   uint64_t q_empty;        // both MMA issuers are done with them (count 2)
-  uint64_t s_full[2];      // per query tile g: S_j landed in TMEM
+  uint64_t s_full[2][2];   // per query tile g and S buffer: S_j landed in TMEM
   uint64_t s_free[2];      // per g: the softmax warps have read S_j
-  uint64_t p_full[2];      // per g: P_j written to TMEM (and O rescaled if needed)
-  uint64_t pv_done[2];     // per g: PV_j finished (P buffer and O are free again)
+  uint64_t p_full[2][2];   // per g and buffer: P_j written to TMEM (and O rescaled if needed)
+  uint64_t pv_done[2][2];  // per g and buffer: PV_j finished (its P buffer is free again)
   uint64_t o_free[2];      // per g: the epilogue has read O of the segment
   uint64_t drain[2];
   uint64_t kv_full[kMaxStages];
@@ -323,15 +328,20 @@ struct Bars {
 
 static_assert(sizeof(Bars) <= 256, "barrier block exceeds its shared-memory slot");
 
-// Tensor-memory columns of query tile g (256 columns at 256 g): S [0,128); head_dim 64:
-// P [128,192), O [192,256); head_dim 128: O [128,256), P written over S [0,64) after S is
-// read into registers.
+// Tensor-memory columns of query tile g (256 columns at 256 g).  head_dim 64 (128-key tiles):
+// S [0,128), P [128,192), O [192,256), one S/P buffer.  head_dim 128 (64-key tiles): two
+// buffers S_b [64 b, 64 b + 64) with P_b written over the first 32 columns of S_b after S_b
+// is read into registers, O [128,256); tile j uses buffer j % 2, so S_{j+1} can be computed
+// while PV_j still reads P_j.
 template <int D>
 struct TmemMap {
-  static constexpr uint32_t S = 0;
-  static constexpr uint32_t P = D == 64 ? 128 : 0;
+  static constexpr int NB = D == 64 ? 1 : 2;  // S/P buffers
+  __host__ __device__ static constexpr uint32_t S(int b) { return D == 64 ? 0 : 64 * b; }
+  __host__ __device__ static constexpr uint32_t P(int b) { return D == 64 ? 128 : 64 * b; }
   static constexpr uint32_t O = D == 64 ? 192 : 128;
-  static constexpr bool kPAliasesS = D != 64;
+  // buffer of tile t, and the phase parity of that buffer's barriers at tile t
+  __device__ static int buf(int t) { return NB == 1 ? 0 : (t & 1); }
+  __device__ static uint32_t par(int t) { return (uint32_t)(NB == 1 ? t : (t >> 1)) & 1u; }
 };
 
 // One run of key tiles of one unit, as a CTA walks its share of the work.
@@ -387,10 +397,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(bars->q_full), 1);
     mbar_init(bar(bars->q_empty), 2);
     for (int g = 0; g < 2; ++g) {
-      mbar_init(bar(bars->s_full[g]), 1);
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(bar(bars->s_full[g][b]), 1);
+        mbar_init(bar(bars->p_full[g][b]), 128);
+        mbar_init(bar(bars->pv_done[g][b]), 1);
+      }
       mbar_init(bar(bars->s_free[g]), 128);
-      mbar_init(bar(bars->p_full[g]), 128);
-      mbar_init(bar(bars->pv_done[g]), 1);
       mbar_init(bar(bars->o_free[g]), 128);
       mbar_init(bar(bars->drain[g]), 1);
     }
@@ -432,11 +444,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const int n_q = seg_nq(p, sg, q_tiles);
       const int head = seg_head(p, sg);
-      mbar_expect_tx(bar(bars->q_full), n_q * C::TILE_BYTES);
+      mbar_expect_tx(bar(bars->q_full), n_q * C::Q_TILE);
       for (int g = 0; g < n_q; ++g) {
 #pragma unroll
         for (int a = 0; a < C::ATOMS; ++a)
-          tma_load_3d(sQ + g * C::TILE_BYTES + a * C::ATOM_BYTES, &p.tm_q, 64 * a, head,
+          tma_load_3d(sQ + g * C::Q_TILE + a * C::Q_ATOM, &p.tm_q, 64 * a, head,
                       (2 * seg_pair(p, sg) + g) * BM, bar(bars->q_full));
       }
       for (int t = sg.a; t < sg.b; ++t, ++issued) {
@@ -447,15 +459,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
-        const TileRef tr = tile_ref(p, t);
+        const TileRef tr = tile_ref<C::BN>(p, t);
         const CUtensorMap* tk = tr.special ? &p.tm_ks : &p.tm_kp;
         const CUtensorMap* tv = tr.special ? &p.tm_vs : &p.tm_vp;
-        mbar_expect_tx(bar(bars->kv_full[s]), 2 * C::TILE_BYTES);
+        mbar_expect_tx(bar(bars->kv_full[s]), 2 * C::KV_TILE);
 #pragma unroll
         for (int a = 0; a < C::ATOMS; ++a) {
-          tma_load_3d(sK + s * C::TILE_BYTES + a * C::ATOM_BYTES, tk, 64 * a, tr.row0, head,
+          tma_load_3d(sK + s * C::KV_TILE + a * C::KV_ATOM, tk, 64 * a, tr.row0, head,
                       bar(bars->kv_full[s]));
-          tma_load_3d(sV + s * C::TILE_BYTES + a * C::ATOM_BYTES, tv, 64 * a, tr.row0, head,
+          tma_load_3d(sV + s * C::KV_TILE + a * C::KV_ATOM, tv, 64 * a, tr.row0, head,
                       bar(bars->kv_full[s]));
         }
       }
@@ -478,12 +490,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1 || warp == 2) {
     // ---------------- MMA issuers: warp 1 for query tile 0, warp 2 for tile 1 ----------------
     const int g = warp - 1;
-    constexpr uint32_t idesc_s = idesc_bf16(BM, BN, false);
+    constexpr uint32_t idesc_s = idesc_bf16(BM, C::BN, false);
     constexpr uint32_t idesc_o = idesc_bf16(BM, D, true);
-    const uint32_t tS = tmem + 256 * g + TM::S;
-    const uint32_t tP = tmem + 256 * g + TM::P;
-    const uint32_t tO = tmem + 256 * g + TM::O;
-    const uint32_t q_base = sQ + g * C::TILE_BYTES;
+    const uint32_t tg = tmem + 256 * g;
+    const uint32_t tO = tg + TM::O;
+    const uint32_t q_base = sQ + g * C::Q_TILE;
     int ring = 0;     // key tiles consumed from the ring (all segments)
     int jg = 0;       // key tiles processed by this query tile (all segments)
     int segs = 0;     // segments this query tile took part in
@@ -518,54 +529,54 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r = ring + (j - j0);
         if (!mbar_wait_warp(bar(bars->kv_full[s]), (r / C::NS) & 1, abort_flag, p.err, 4))
           return false;
-        if (j >= 1 && !mbar_wait_warp(bar(bars->s_free[g]), (j - 1) & 1, abort_flag, p.err, 5))
+        // the S buffer of tile j is free: one buffer, the softmax has read S_{j-1}; two
+        // buffers, PV_{j-2} has read P_{j-2}, which was written after S_{j-2} was read
+        if (TM::NB == 1) {
+          if (j >= 1 &&
+              !mbar_wait_warp(bar(bars->s_free[g]), (j - 1) & 1, abort_flag, p.err, 5))
+            return false;
+        } else if (j >= 2 && !mbar_wait_warp(bar(bars->pv_done[g][TM::buf(j)]), TM::par(j - 2),
+                                             abort_flag, p.err, 5)) {
           return false;
+        }
         tc_fence_after();
-        const uint32_t k_base = sK + s * C::TILE_BYTES;
+        const uint32_t k_base = sK + s * C::KV_TILE;
+        const uint32_t tS = tg + TM::S(TM::buf(j));
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::ATOM_BYTES + (kk & 3) * 32;
-          mma_ss(tS, sdesc(q_base + off, 16, 1024), sdesc(k_base + off, 16, 1024), idesc_s,
+          const uint32_t qo = (kk >> 2) * C::Q_ATOM + (kk & 3) * 32;
+          const uint32_t ko = (kk >> 2) * C::KV_ATOM + (kk & 3) * 32;
+          mma_ss(tS, sdesc(q_base + qo, 16, 1024), sdesc(k_base + ko, 16, 1024), idesc_s,
                  kk > 0 ? 1u : 0u);
         }
-        mma_commit(bar(bars->s_full[g]));
+        mma_commit(bar(bars->s_full[g][TM::buf(j)]));
         return true;
       };
       auto issue_pv = [&](int i) -> bool {
-        if (!mbar_wait_warp(bar(bars->p_full[g]), i & 1, abort_flag, p.err, 3)) return false;
+        if (!mbar_wait_warp(bar(bars->p_full[g][TM::buf(i)]), TM::par(i), abort_flag, p.err, 3))
+          return false;
         // O of the previous segment must have been read out before the first PV overwrites it
         if (i == j0 && segs > 0 &&
             !mbar_wait_warp(bar(bars->o_free[g]), (segs - 1) & 1, abort_flag, p.err, 13))
           return false;
         tc_fence_after();
         const int s = (ring + (i - j0)) % C::NS;
-        const uint32_t v_base = sV + s * C::TILE_BYTES;
+        const uint32_t v_base = sV + s * C::KV_TILE;
+        const uint32_t tP = tg + TM::P(TM::buf(i));
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          // B = V tile [keys][D], MN-major: 16 keys = 2 groups of 8 rows of 128 B
-          const uint64_t bd = sdesc(v_base + kk * 2048, C::ATOM_BYTES, 1024);
+        for (int kk = 0; kk < C::BN / 16; ++kk) {
+          // B = V tile [keys][D], MN-major: 16 keys = 2 groups of 8 rows of 128 B; the next
+          // 64 features are one atom column (KV_ATOM bytes) further
+          const uint64_t bd = sdesc(v_base + kk * 2048, C::KV_ATOM, 1024);
           mma_ts(tO, tP + 8 * kk, bd, idesc_o, (i > j0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit(bar(bars->pv_done[g]));
+        mma_commit(bar(bars->pv_done[g][TM::buf(i)]));
         mma_commit(bar(bars->kv_empty[s]));
         return true;
       };
-      // with P written over S, the previous segment's last PV must have read P before the
-      // first S of this segment overwrites it
-      if (TM::kPAliasesS && j0 > 0)
-        ok = mbar_wait_warp(bar(bars->pv_done[g]), (j0 - 1) & 1, abort_flag, p.err, 14);
+      // S_j is issued before PV_{j-1}, so the softmax can start on it early
       ok = ok && issue_qk(j0);
-      for (int j = j0 + 1; ok && j < j0 + n; ++j) {
-        if (TM::kPAliasesS) {
-          // P_{j-1} lives in S: PV_{j-1} must have read it before S_j overwrites it
-          ok = issue_pv(j - 1) &&
-               mbar_wait_warp(bar(bars->pv_done[g]), (j - 1) & 1, abort_flag, p.err, 10) &&
-               issue_qk(j);
-        } else {
-          // S_j only needs S_{j-1} read: issue it first so the softmax can start early
-          ok = issue_qk(j) && issue_pv(j - 1);
-        }
-      }
+      for (int j = j0 + 1; ok && j < j0 + n; ++j) ok = issue_qk(j) && issue_pv(j - 1);
       if (ok) {
         // the last QK of the segment has been issued: the query buffers can be refilled once
         // it completes
@@ -587,9 +598,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quad = warp & 3;                  // TMEM lane quadrant this warp may access
     const int row_in_pair = g * BM + quad * 32 + lane;
     const uint32_t lane_base = tmem + 256 * g + ((uint32_t)(quad * 32) << 16);
-    const uint32_t tS = lane_base + TM::S;
-    const uint32_t tP = lane_base + TM::P;
     const uint32_t tO = lane_base + TM::O;
+    constexpr int BN = C::BN;
     int jg = 0;
     int seg_i = 0;
     bool ok = true;
@@ -605,7 +615,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = j0; ok && j < j0 + n; ++j) {
         // every wait in these warps is made warp-uniform, so warp-collective tcgen05 ops and
         // votes below always run with the whole warp
-        if (!__all_sync(kFull, mbar_wait(bar(bars->s_full[g]), j & 1, abort_flag, p.err, 6))) {
+        const int sb = TM::buf(j);
+        const uint32_t tS = lane_base + TM::S(sb);
+        const uint32_t tP = lane_base + TM::P(sb);
+        if (!__all_sync(kFull, mbar_wait(bar(bars->s_full[g][sb]), TM::par(j), abort_flag, p.err,
+                                         6))) {
           ok = false;
           break;
         }
@@ -617,7 +631,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         mbar_arrive(bar(bars->s_free[g]));
 
-        const int valid = tile_ref(p, sg.a + (j - j0)).valid;
+        const int valid = tile_ref<BN>(p, sg.a + (j - j0)).valid;
         if (valid != BN) {
           // keys past the end of a page / of the special stream: -inf scores, zero weight
 #pragma unroll
@@ -643,9 +657,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           l *= alpha;
           rescale = true;
         }
-        // P_j overwrites P_{j-1} (and O may be rescaled): PV_{j-1} must have finished
-        if (j >= 1 && !__all_sync(kFull, mbar_wait(bar(bars->pv_done[g]), (j - 1) & 1,
-                                                   abort_flag, p.err, 7))) {
+        // one P buffer: P_j overwrites P_{j-1}, so PV_{j-1} must have finished (two buffers:
+        // P_j goes to its own S buffer; PV_{j-1} is waited for only before rescaling O)
+        if (TM::NB == 1 && j >= 1 &&
+            !__all_sync(kFull, mbar_wait(bar(bars->pv_done[g][0]), (j - 1) & 1, abort_flag,
+                                         p.err, 7))) {
           ok = false;
           break;
         }
@@ -680,6 +696,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (__any_sync(kFull, rescale) && j > j0) {
           // O holds sum_{i<j} P_i V_i relative to the old max: scale it before PV_j lands
+          if (TM::NB == 2 &&
+              !__all_sync(kFull, mbar_wait(bar(bars->pv_done[g][TM::buf(j - 1)]),
+                                           TM::par(j - 1), abort_flag, p.err, 7))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
@@ -694,11 +717,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(bars->p_full[g]));
+        mbar_arrive(bar(bars->p_full[g][sb]));
       }
       jg += n;
       if (!ok ||
-          !__all_sync(kFull, mbar_wait(bar(bars->pv_done[g]), (jg - 1) & 1, abort_flag, p.err,
+          !__all_sync(kFull, mbar_wait(bar(bars->pv_done[g][TM::buf(jg - 1)]), TM::par(jg - 1),
+                                       abort_flag, p.err,
                                        9))) {
         ok = false;
         break;

@@ -57,7 +57,7 @@ struct lbm_cache {
 
 namespace {
 
-constexpr int kKeyTile = 128;  // keys per attention key tile (page strides are multiples)
+constexpr int kKeyTile = 128;  // page strides are multiples (of every attention key tile)
 
 int elem_size(int dtype) { return dtype == LBM_BF16 ? 2 : 4; }
 
@@ -138,10 +138,11 @@ int fill_attn_params(lbm_cache* c, int block, const void* q, void* out, lbm::Att
   p.heads = c->heads;
   p.patches = c->patches;
   p.page_stride = bk.pools.page_stride;
-  p.tiles_per_page = (c->patches + kKeyTile - 1) / kKeyTile;
+  const int kt = lbm::attn_key_tile(c->head_dim);  // keys per attention key tile
+  p.tiles_per_page = (c->patches + kt - 1) / kt;
   p.n_pages = n_pages;
   p.n_special = n_sp;
-  p.n_tiles = p.n_pages * p.tiles_per_page + (n_sp + kKeyTile - 1) / kKeyTile;
+  p.n_tiles = p.n_pages * p.tiles_per_page + (n_sp + kt - 1) / kt;
   p.n_pairs = ((T + 127) / 128 + 1) / 2;
   p.work = (long long)p.n_pairs * c->heads * p.n_tiles;
   if (p.work >= (1LL << 31)) return LBM_ERR_UNSUPPORTED;  // the kernel counts in 32 bits
@@ -360,7 +361,7 @@ int lbm_cache_create_blocks(int num_blocks, int heads, int head_dim, int patches
   if (dtype == LBM_BF16) {
     const uint64_t row = (uint64_t)head_dim * 2;
     const uint64_t prow = (uint64_t)P * stride;
-    const uint32_t kt = kKeyTile;
+    const uint32_t kt = (uint32_t)lbm::attn_key_tile(head_dim);  // tensor-map box rows
     for (CacheBlock& bk : c->blocks) {
       const lbm::Pools& pl = bk.pools;
       if (!make_map(&bk.tm_kp, pl.k_patch, head_dim, prow, heads, row, prow * row, kt, 1) ||

@@ -43,6 +43,11 @@ struct AppendArgs {
 
 constexpr int kMaxPages = 1024;
 
+// Keys per K/V tile of the tensor-core attention: 128 at head_dim 64; 64 at head_dim 128,
+// where two score buffers of a query tile then fit next to its 128 output columns in tensor
+// memory.  Host (tile counts, tensor-map boxes) and kernel use this one definition.
+__host__ __device__ constexpr int attn_key_tile(int head_dim) { return head_dim == 64 ? 128 : 64; }
+
 constexpr int kMaxGrid = 1024;  // persistent attention CTAs per launch, at most
 
 // Kernel parameter block of the paged attention (passed by value).
