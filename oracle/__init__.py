@@ -15,10 +15,13 @@ cited by title and section:
 * [RealTime3D] "How LingBot-Map Achieves Real-Time 3D Reconstruction: Streaming Transformers
                and KV Caching"
 * [KVBenefits] "KV Caching Benefits in Ling Bot-Map: 7 Advantages for Streaming Vision Models"
+* [RoPERange]  "How to Handle Sequences Exceeding the RoPE Training Range in LingBot-Map"
 
 Modules:
 
 * ``rope3d``     per-axis frequency tables, token positions, rotation (fp64).
+* ``rope2d``     the 2D (y, x) variant: halves of the features per axis, base frequency
+                 100, tables sized from the token count.
 * ``retention``  the page table / free list / deferred-eviction state machine, plus the
                  closed form of the retained set.
 * ``attention``  explicit masked softmax attention over the whole history, and over the
@@ -35,4 +38,4 @@ order, special page size): those are stated readings, self-consistent across ora
 CUDA path.
 """
 
-from . import rope3d, retention, attention, stream  # noqa: F401
+from . import rope3d, rope2d, retention, attention, stream  # noqa: F401

@@ -65,19 +65,6 @@ def inv_freq(d_axis: int, theta: float = THETA, ntk_factor: float = 1.0) -> np.n
     return base ** (-(2.0 * i) / float(d_axis))
 
 
-def axis_tables(head_dim: int, n_t: int, n_h: int, n_w: int, theta: float = THETA,
-                split=None, ntk_factor: float = 1.0):
-    """Per-axis angle tables: ang_t[n_t, d_t/2], ang_h[n_h, d_h/2], ang_w[n_w, d_w/2].
-
-    Row p of an axis table holds p * inv_freq of that axis (fp64 angles in radians).
-    """
-    d_t, d_h, d_w = axis_split(head_dim, split)
-    ang_t = np.outer(np.arange(n_t, dtype=np.float64), inv_freq(d_t, theta, ntk_factor))
-    ang_h = np.outer(np.arange(n_h, dtype=np.float64), inv_freq(d_h, theta, ntk_factor))
-    ang_w = np.outer(np.arange(n_w, dtype=np.float64), inv_freq(d_w, theta, ntk_factor))
-    return ang_t, ang_h, ang_w
-
-
 def token_positions(frame_idx: int, patch_start_idx: int, pph: int, ppw: int) -> np.ndarray:
     """(t, h, w) of every token of one frame, shape [patch_start_idx + pph*ppw, 3], int64.
 

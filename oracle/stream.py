@@ -22,7 +22,7 @@ from dataclasses import dataclass
 
 import numpy as np
 
-from . import attention, retention, rope3d
+from . import attention, retention, rope2d, rope3d
 
 ROW_CHUNK = 64
 
@@ -48,12 +48,15 @@ class StreamOracle:
     def __init__(self, heads: int, head_dim: int, pph: int, ppw: int, scale_frames: int,
                  sliding_window: int, max_frames: int, specials_per_frame: int = 6,
                  theta: float = rope3d.THETA, keep_history: bool = False, kv_source=None,
-                 split=None, ntk_factor: float = 1.0):
+                 split=None, ntk_factor: float = 1.0, rope2d_frequency: float | None = None):
         """split / ntk_factor: an explicit (t, h, w) feature split and NTK factor of the 3D
-        RoPE (``rope3d.axis_split``, ``rope3d.inv_freq``).  kv_source, if given, is a callable (frame, region) -> (k, v) returning a past
-        frame's unrotated inputs (region "patch": [pph*ppw, H, D], "special": [6, H, D]);
-        the oracle then keeps no K/V of its own and re-creates retained keys when a frame
-        attends, which keeps long streams small in memory."""
+        RoPE (``rope3d.axis_split``, ``rope3d.inv_freq``).  rope2d_frequency: rotate with the
+        2D (y, x) embedding of that base frequency instead (``rope2d``; the frame index then
+        plays no part in the rotation).  kv_source, if given, is a callable
+        (frame, region) -> (k, v) returning a past frame's unrotated inputs (region "patch":
+        [pph*ppw, H, D], "special": [6, H, D]); the oracle then keeps no K/V of its own and
+        re-creates retained keys when a frame attends, which keeps long streams small in
+        memory."""
         self.heads = heads
         self.head_dim = head_dim
         self.pph = pph
@@ -62,6 +65,7 @@ class StreamOracle:
         self.theta = theta
         self.split = split
         self.ntk_factor = ntk_factor
+        self.rope2d_frequency = rope2d_frequency
         self.ret = retention.PagedRetention(scale_frames, sliding_window, max_frames,
                                             specials_per_frame)
         self.patch_kv: dict = {}      # frame -> (k [Pf,H,D], v [Pf,H,D]) of retained frames
@@ -90,21 +94,27 @@ class StreamOracle:
                     return ks, vs
             raise KeyError(frame)
         k, v = self.kv_source(frame, region)
+        ang = self.angles(frame)
+        ang = ang[self.psi:] if region == "patch" else ang[:self.psi]
+        return rope3d.rotate(k, ang), np.asarray(v, dtype=np.float64)
+
+    def angles(self, frame: int) -> np.ndarray:
+        """Rotation angles of every token of frame ``frame``: [T, head_dim / 2]."""
+        if self.rope2d_frequency is not None:
+            pos = rope2d.token_positions(self.psi, self.pph, self.ppw)
+            return rope2d.angles_for_positions(pos, self.head_dim, self.rope2d_frequency)
         pos = rope3d.token_positions(frame, self.psi, self.pph, self.ppw)
-        pos = pos[self.psi:] if region == "patch" else pos[:self.psi]
-        kr = rope3d.rotate(k, rope3d.angles_for_positions(pos, self.head_dim, self.theta,
-                                                                self.split, self.ntk_factor))
-        return kr, np.asarray(v, dtype=np.float64)
+        return rope3d.angles_for_positions(pos, self.head_dim, self.theta, self.split,
+                                           self.ntk_factor)
 
     def step(self, frame_idx: int, is_keyframe: bool, q: np.ndarray, k: np.ndarray,
              v: np.ndarray, rows=None, attend: bool = True) -> FrameResult:
         T = self.tokens_per_frame
         assert q.shape == (T, self.heads, self.head_dim), q.shape
         page, slot = self.ret.append(frame_idx, is_keyframe)
-        qr = rope3d.rotate_frame(q, frame_idx, self.psi, self.pph, self.ppw, self.theta,
-                                 self.split, self.ntk_factor)
-        kr = rope3d.rotate_frame(k, frame_idx, self.psi, self.pph, self.ppw, self.theta,
-                                 self.split, self.ntk_factor)
+        ang = self.angles(frame_idx)
+        qr = rope3d.rotate(q, ang)
+        kr = rope3d.rotate(k, ang)
         v64 = np.asarray(v, dtype=np.float64)
         vis = self.ret.visible()
 

@@ -121,3 +121,36 @@ def test_split_axes_swapped_is_caught(monkeypatch):
         return d_h, d_t, d_w
     monkeypatch.setattr(rope3d, "axis_split", bad_split)
     _fails(tp.test_each_axis_is_library_1d_rope, 64, "example_fhw_dim", 1.0)
+
+
+# ---- the 2D variant ("How to Handle Sequences Exceeding the RoPE Training Range in
+# LingBot-Map") ----
+
+import test_oracle_rope2d as t2  # noqa: E402
+from oracle import rope2d  # noqa: E402
+
+
+def test_rope2d_halves_swapped_is_caught(monkeypatch):
+    orig = rope2d.angles_for_positions
+
+    def bad(pos, head_dim, frequency=rope2d.FREQUENCY, seq_len=None):
+        return orig(np.asarray(pos)[:, ::-1], head_dim, frequency, seq_len)   # x half first
+    monkeypatch.setattr(rope2d, "angles_for_positions", bad)
+    _fails(t2.test_each_half_is_library_1d_rope, 64)
+
+
+def test_rope2d_base_of_the_3d_axes_is_caught(monkeypatch):
+    orig = rope2d.inv_freq
+
+    def bad(d_half, frequency=rope2d.FREQUENCY):
+        return orig(d_half, 10000.0)                   # the 3D embedding's theta
+    monkeypatch.setattr(rope2d, "inv_freq", bad)
+    _fails(t2.test_each_half_is_library_1d_rope, 128)
+
+
+def test_rope2d_table_sized_by_max_position_is_caught(monkeypatch):
+    def bad(d_half, seq_len, frequency=rope2d.FREQUENCY):
+        ang = np.outer(np.arange(65, dtype=np.float64), rope2d.inv_freq(d_half, frequency))
+        return np.cos(ang), np.sin(ang)                # max position + 1 rows (64x64 grid)
+    monkeypatch.setattr(rope2d, "frequency_components", bad)
+    _fails(t2.test_page_example_shapes)
