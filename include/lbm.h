@@ -12,6 +12,7 @@
  *                 Transformers and KV Caching"
  *   [KVBenefits] "KV Caching Benefits in Ling Bot-Map: 7 Advantages for Streaming Vision
  *                 Models"
+ *   [RoPERange]  "How to Handle Sequences Exceeding the RoPE Training Range in LingBot-Map"
  *
  * Conventions common to every call
  * --------------------------------
@@ -88,19 +89,51 @@ typedef struct lbm_pager lbm_pager_t;
 LBM_API int lbm_rope3d_tables(int head_dim, int ppf, int pph, int ppw, int patch_start_idx,
                       double theta, lbm_rope_t** out);
 
-/* Writes the expanded table of [3DRoPE-KV] "Multi-Axis Frequency Generation": cos and sin,
- * each float [ppf * (patch_start_idx + pph*ppw)][head_dim/2] (device pointers, caller-owned),
- * frames 0..ppf-1 in order, tokens of a frame in the order above.  Enqueued on stream. */
 /* The same tables with an explicit (t, h, w) split of head_dim = d_t + d_h + d_w (the pages'
  * fhw_dim, e.g. [20, 22, 22] for head_dim 64 in [3DRoPE-KV] "Implementation Example" and
  * [40, 44, 44] for 128 in [VideoRoPE] "Enabling 3D RoPE for Video Heads") and an NTK factor
- * that multiplies theta ([VideoRoPE] "NTK-Aware Frequency Scaling").  Each axis size even and
- * >= 2, ntk_factor > 0, theta * ntk_factor > 1; otherwise LBM_ERR_INVALID.  lbm_rope3d_tables
- * is this call with the default split and ntk_factor 1. */
-LBM_API int lbm_rope3d_tables_fhw(int d_t, int d_h, int d_w, int ppf, int pph, int ppw,
-                                  int patch_start_idx, double theta, double ntk_factor,
+ * that multiplies theta ([VideoRoPE] "NTK-Aware Frequency Scaling").
+ *   head_dim       even, >= 6
+ *   d_t, d_h, d_w  each even and >= 2, summing to head_dim; or all three 0 for the default
+ *                  split of lbm_rope3d_tables (d_h = d_w = 2*(head_dim/6), d_t = the rest)
+ *   ntk_factor     > 0, with theta * ntk_factor > 1
+ * Otherwise LBM_ERR_INVALID.  lbm_rope3d_tables is this call with the default split and
+ * ntk_factor 1.  Allocates device memory on the current device; synchronous. */
+LBM_API int lbm_rope3d_tables_fhw(int head_dim, int d_t, int d_h, int d_w, int ppf, int pph,
+                                  int ppw, int patch_start_idx, double theta, double ntk_factor,
                                   lbm_rope_t** out);
 
+/* The 2D (y, x) variant of [RoPERange] "How to Handle Sequences Exceeding the RoPE Training
+ * Range in LingBot-Map", sections "Spatial Position Encoding" and "Dynamic Frequency Caching
+ * for Arbitrary Sequence Lengths": the features split into two halves of head_dim/2, the
+ * first rotated by a 1D rotary embedding of the row y, the second by one of the column x,
+ * angle(p, i) = p * frequency^(-2i/(head_dim/2)), i < head_dim/4, frequency 100.0 on the
+ * page; each half's table has one row per token of a frame (sized from the token count, not
+ * from the largest coordinate).  Token j of a frame sits at (0, 0) for j < patch_start_idx and
+ * at (1 + r, 1 + c) for patch (r, c); the frame index plays no part in the rotation (frames
+ * are still told apart by the cache).  Feature pair i is (x[2i], x[2i+1]); pairs
+ * [0, head_dim/4) take y, the rest x.  The page's scaling_factor (1.0, undefined there) is not
+ * modelled.
+ *   head_dim       a multiple of 4 (caches take 64 / 128)
+ *   ppf            frames a cache using these tables may stream (frame_idx < ppf)
+ *   pph, ppw, patch_start_idx   as for lbm_rope3d_tables
+ *   frequency      > 1
+ * The result is used exactly like a 3D table object (caches, lbm_rope3d_expand,
+ * lbm_rope_destroy).  LBM_ERR_INVALID for bad sizes.  Allocates device memory on the
+ * current device; synchronous. */
+LBM_API int lbm_rope2d_tables(int head_dim, int ppf, int pph, int ppw, int patch_start_idx,
+                              double frequency, lbm_rope_t** out);
+
+/* Writes the expanded table of [3DRoPE-KV] "Multi-Axis Frequency Generation" (the one the
+ * page prints as [ppf * (patch_start_idx + pph*ppw)][head_dim/2]), for parity checks of the
+ * tables a rope object holds.
+ *   rope            from lbm_rope3d_tables / lbm_rope3d_tables_fhw / lbm_rope2d_tables
+ *   cos_out, sin_out  DEVICE pointers, caller-owned, float [ppf * (patch_start_idx +
+ *                  pph*ppw)][head_dim/2] each: row = frame * tokens_per_frame + token, frames
+ *                  0..ppf-1 in order, a frame's tokens in the order above (specials, then
+ *                  patches row-major); column = feature pair
+ *   stream          cudaStream_t the kernel is enqueued on (nothing waits for it)
+ * LBM_ERR_INVALID for a null argument, LBM_ERR_CUDA if the launch fails. */
 LBM_API int lbm_rope3d_expand(const lbm_rope_t* rope, float* cos_out, float* sin_out, void* stream);
 
 LBM_API void lbm_rope_destroy(lbm_rope_t* rope);
@@ -202,7 +235,12 @@ LBM_API int lbm_commit_frame(lbm_cache_t* cache, int keep);
  * instead of the cache's own scratch; the call allocates nothing (device or host heap).
  *   - bf16 caches only (LBM_ERR_UNSUPPORTED otherwise).
  *   - The first call on a device looks up the array's device address with that device
- *     current; make that first call before any stream capture.
+ *     current; make that first call before any stream capture.  Host threads may make their
+ *     first calls at the same time (the lookup is guarded), but calls on one cache must not
+ *     run concurrently, as for every call on a cache.
+ *   - With one CTA per SM (148 on a B200): a head_dim 64 frame fits while units + 148 <= 252
+ *     (16 heads: up to 12 query tiles, 1536 tokens); a head_dim 128 frame whose keys are
+ *     split needs at least 149 x 256 x 129 x 4 bytes (19.5 MB) and is always refused.
  *   - A frame whose units are shared by CTAs and whose partial results need more than
  *     LBM_NOALLOC_SCRATCH_BYTES ((units + CTAs) x 256 x (head_dim + 1) x 4 bytes) is refused
  *     with LBM_ERR_CAPACITY and the cache is left as it was.

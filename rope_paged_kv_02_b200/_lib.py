@@ -32,7 +32,8 @@ LBM_MAX_PAGES = 1024
 
 # every symbol include/lbm.h declares
 SYMBOLS = [
-    "lbm_rope3d_tables", "lbm_rope3d_tables_fhw", "lbm_rope3d_expand", "lbm_rope_destroy",
+    "lbm_rope3d_tables", "lbm_rope3d_tables_fhw", "lbm_rope2d_tables", "lbm_rope3d_expand",
+    "lbm_rope_destroy",
     "lbm_cache_create", "lbm_cache_create_blocks", "lbm_append_frame", "lbm_append_frame_block",
     "lbm_attend_frame", "lbm_attend_frame_block", "lbm_attend_frame_noalloc",
     "lbm_commit_frame", "lbm_cache_reset", "lbm_cache_read_kv_block",
@@ -91,7 +92,8 @@ def load() -> ctypes.CDLL:
     c_int, c_ll, c_void, c_d = ctypes.c_int, ctypes.c_longlong, ctypes.c_void_p, ctypes.c_double
     pint = ctypes.POINTER(c_int)
     lib.lbm_rope3d_tables.argtypes = [c_int] * 5 + [c_d, ctypes.POINTER(c_void)]
-    lib.lbm_rope3d_tables_fhw.argtypes = [c_int] * 7 + [c_d, c_d, ctypes.POINTER(c_void)]
+    lib.lbm_rope3d_tables_fhw.argtypes = [c_int] * 8 + [c_d, c_d, ctypes.POINTER(c_void)]
+    lib.lbm_rope2d_tables.argtypes = [c_int] * 5 + [c_d, ctypes.POINTER(c_void)]
     lib.lbm_rope3d_expand.argtypes = [c_void, c_void, c_void, c_void]
     lib.lbm_rope_destroy.argtypes = [c_void]
     lib.lbm_rope_destroy.restype = None
@@ -185,22 +187,18 @@ class Rope3D:
 
     def __init__(self, head_dim: int, ppf: int, pph: int, ppw: int, patch_start_idx: int = 6,
                  theta: float = 10000.0, split=None, ntk_factor: float = 1.0):
-        """split: explicit (d_t, d_h, d_w) summing to head_dim (lbm_rope3d_tables_fhw)."""
+        """split: explicit (d_t, d_h, d_w) summing to head_dim (lbm_rope3d_tables_fhw);
+        None leaves the split to the library's default."""
         lib = load()
         h = ctypes.c_void_p()
         if split is None and ntk_factor == 1.0:
             _check(lib.lbm_rope3d_tables(head_dim, ppf, pph, ppw, patch_start_idx, theta,
                                          ctypes.byref(h)), "lbm_rope3d_tables")
         else:
-            if split is None:
-                dh = 2 * (head_dim // 6)
-                split = (head_dim - 2 * dh, dh, dh)
-            if sum(split) != head_dim:
-                raise ValueError("split must sum to head_dim")
-            _check(lib.lbm_rope3d_tables_fhw(int(split[0]), int(split[1]), int(split[2]), ppf,
-                                             pph, ppw, patch_start_idx, theta,
-                                             float(ntk_factor), ctypes.byref(h)),
-                   "lbm_rope3d_tables_fhw")
+            d_t, d_h, d_w = (0, 0, 0) if split is None else (int(x) for x in split)
+            _check(lib.lbm_rope3d_tables_fhw(head_dim, d_t, d_h, d_w, ppf, pph, ppw,
+                                             patch_start_idx, theta, float(ntk_factor),
+                                             ctypes.byref(h)), "lbm_rope3d_tables_fhw")
         self.handle = h
         self.head_dim, self.ppf, self.pph, self.ppw = head_dim, ppf, pph, ppw
         self.patch_start_idx = patch_start_idx
@@ -220,6 +218,20 @@ class Rope3D:
             self.close()
         except Exception:
             pass
+
+
+class Rope2D(Rope3D):
+    """lbm_rope2d_tables: the 2D (y, x) variant's tables (device), built once; used like
+    Rope3D by caches."""
+
+    def __init__(self, head_dim: int, ppf: int, pph: int, ppw: int, patch_start_idx: int = 6,
+                 frequency: float = 100.0):
+        h = ctypes.c_void_p()
+        _check(load().lbm_rope2d_tables(head_dim, ppf, pph, ppw, patch_start_idx,
+                                        float(frequency), ctypes.byref(h)), "lbm_rope2d_tables")
+        self.handle = h
+        self.head_dim, self.ppf, self.pph, self.ppw = head_dim, ppf, pph, ppw
+        self.patch_start_idx = patch_start_idx
 
 
 class PagedKVCache:

@@ -10,6 +10,9 @@
 // The array is shared by every call on a device and keeps the last call's contents.  No
 // part of it needs to start at zero: each call writes every partial row it later reads.
 // Calls that overlap on the GPU (two streams, or two caches at once) race on it.
+#include <atomic>
+#include <mutex>
+
 #include "../../include/lbm.h"
 #include "lbm_internal.h"
 
@@ -20,9 +23,14 @@ constexpr size_t kNoallocScratchFloats = LBM_NOALLOC_SCRATCH_BYTES / sizeof(floa
 
 static __device__ __align__(256) float g_noalloc_scratch[kNoallocScratchFloats];
 
+// Device address of the array, per device, once looked up.  In host code the array's name
+// is only a host-side stand-in: the address a kernel may be given comes from
+// cudaGetSymbolAddress with that device current.  Host threads may make their first call on a
+// device at the same time: the lookup runs under a mutex, the result is published with
+// release / acquire order.
 constexpr int kMaxDevices = 64;
-float* g_scratch_ptr[kMaxDevices];  // device address of the array, per device, once set
-bool g_scratch_ready[kMaxDevices];
+std::atomic<float*> g_scratch_ptr[kMaxDevices];
+std::mutex g_scratch_lookup;
 
 }  // namespace
 
@@ -30,16 +38,21 @@ bool g_scratch_ready[kMaxDevices];
 // first call on a device looks the address up (cudaGetSymbolAddress) and remembers it.
 int noalloc_scratch(int device, float** ptr, size_t* floats) {
   if (device < 0 || device >= kMaxDevices || !ptr || !floats) return LBM_ERR_INVALID;
-  if (!g_scratch_ready[device]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
-      cudaGetLastError();
-      return LBM_ERR_CUDA;
+  float* p = g_scratch_ptr[device].load(std::memory_order_acquire);
+  if (!p) {
+    std::lock_guard<std::mutex> lock(g_scratch_lookup);
+    p = g_scratch_ptr[device].load(std::memory_order_relaxed);
+    if (!p) {
+      void* addr = nullptr;
+      if (cudaGetSymbolAddress(&addr, g_noalloc_scratch) != cudaSuccess || !addr) {
+        cudaGetLastError();
+        return LBM_ERR_CUDA;
+      }
+      p = static_cast<float*>(addr);
+      g_scratch_ptr[device].store(p, std::memory_order_release);
     }
-    g_scratch_ptr[device] = static_cast<float*>(p);
-    g_scratch_ready[device] = true;
   }
-  *ptr = g_scratch_ptr[device];
+  *ptr = p;
   *floats = kNoallocScratchFloats;
   return LBM_OK;
 }

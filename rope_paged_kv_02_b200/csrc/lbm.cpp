@@ -164,71 +164,36 @@ void block_attended(lbm_cache* c) {
   }
 }
 
-}  // namespace
+// One axis of a rope object: a table of `rows` positions for the feature pairs of d_axis
+// features, angle(p, i) = p * base^(-2i / d_axis).
+struct AxisSpec {
+  int rows;
+  int d_axis;
+  double base;
+};
 
-extern "C" {
-
-const char* lbm_status_string(int status) {
-  switch (status) {
-    case LBM_OK: return "ok";
-    case LBM_ERR_INVALID: return "invalid argument";
-    case LBM_ERR_UNSUPPORTED: return "unsupported configuration";
-    case LBM_ERR_SEQUENCE: return "call out of sequence";
-    case LBM_ERR_CAPACITY: return "capacity exceeded";
-    case LBM_ERR_NOMEM: return "out of memory";
-    case LBM_ERR_CUDA: return "CUDA error";
-    case LBM_ERR_TIMEOUT: return "device wait timed out";
-    default: return "unknown status";
-  }
-}
-
-int lbm_rope3d_tables(int head_dim, int ppf, int pph, int ppw, int patch_start_idx,
-                      double theta, lbm_rope_t** out) {
-  if (!out) return LBM_ERR_INVALID;
-  *out = nullptr;
-  if (head_dim < 6 || head_dim % 2) return LBM_ERR_INVALID;
-  // Axis split: d_h = d_w = 2 * (head_dim / 6), d_t = the rest; pairs ordered t, h, w.
-  const int dh = 2 * (head_dim / 6);
-  return lbm_rope3d_tables_fhw(head_dim - 2 * dh, dh, dh, ppf, pph, ppw, patch_start_idx, theta,
-                               1.0, out);
-}
-
-int lbm_rope3d_tables_fhw(int dt, int dh, int dw, int ppf, int pph, int ppw,
-                          int patch_start_idx, double theta, double ntk_factor,
-                          lbm_rope_t** out) {
-  if (!out) return LBM_ERR_INVALID;
-  *out = nullptr;
-  if (dt < 2 || dh < 2 || dw < 2 || dt % 2 || dh % 2 || dw % 2 || ppf < 1 || pph < 1 ||
-      ppw < 1 || patch_start_idx < 0 || !(ntk_factor > 0.0) || !(theta * ntk_factor > 1.0) ||
-      (long long)pph * ppw > (1 << 20) || ppf > (1 << 24))
-    return LBM_ERR_INVALID;
-  const int head_dim = dt + dh + dw;
-  theta *= ntk_factor;  // [VideoRoPE] "NTK-Aware Frequency Scaling": theta * ntk_factor
-  lbm::RopeTables t{};
-  t.head_dim = head_dim;
-  t.ppf = ppf;
-  t.pph = pph;
-  t.ppw = ppw;
-  t.psi = patch_start_idx;
-  t.nt = dt / 2;
-  t.nh = dh / 2;
-  t.nw = dw / 2;
-  const size_t n_t = (size_t)ppf * t.nt, n_h = (size_t)(pph + 1) * t.nh,
-               n_w = (size_t)(ppw + 1) * t.nw;
-  std::vector<float2> host(n_t + n_h + n_w);
-  // angle(p, i) = p * theta^(-2i/d_axis), in double, cos/sin rounded once to float
-  auto fill = [&](float2* dst, int rows, int pairs, int d_axis) {
+// Fills the t, h and w tables (angles in double, cos/sin rounded once to float), uploads them
+// and returns the rope object.  An axis with d_axis 0 has no pairs (the 2D variant's t).
+int build_rope(lbm::RopeTables t, AxisSpec at, AxisSpec ah, AxisSpec aw, lbm_rope_t** out) {
+  t.nt = at.d_axis / 2;
+  t.nh = ah.d_axis / 2;
+  t.nw = aw.d_axis / 2;
+  const size_t n_t = (size_t)at.rows * t.nt, n_h = (size_t)ah.rows * t.nh,
+               n_w = (size_t)aw.rows * t.nw;
+  std::vector<float2> host(std::max<size_t>(n_t + n_h + n_w, 1));
+  auto fill = [&](float2* dst, const AxisSpec& ax) {
+    const int pairs = ax.d_axis / 2;
     for (int i = 0; i < pairs; ++i) {
-      const double inv = std::pow(theta, -(2.0 * i) / (double)d_axis);
-      for (int p = 0; p < rows; ++p) {
+      const double inv = std::pow(ax.base, -(2.0 * i) / (double)ax.d_axis);
+      for (int p = 0; p < ax.rows; ++p) {
         const double a = (double)p * inv;
         dst[(size_t)p * pairs + i] = make_float2((float)std::cos(a), (float)std::sin(a));
       }
     }
   };
-  fill(host.data(), ppf, t.nt, dt);
-  fill(host.data() + n_t, pph + 1, t.nh, dh);
-  fill(host.data() + n_t + n_h, ppw + 1, t.nw, dw);
+  fill(host.data(), at);
+  fill(host.data() + n_t, ah);
+  fill(host.data() + n_t + n_h, aw);
   auto* r = new (std::nothrow) lbm_rope;
   if (!r) return LBM_ERR_NOMEM;
   if (cudaGetDevice(&r->device) != cudaSuccess ||
@@ -249,6 +214,78 @@ int lbm_rope3d_tables_fhw(int dt, int dh, int dw, int ppf, int pph, int ppw,
   r->t = t;
   *out = r;
   return LBM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* lbm_status_string(int status) {
+  switch (status) {
+    case LBM_OK: return "ok";
+    case LBM_ERR_INVALID: return "invalid argument";
+    case LBM_ERR_UNSUPPORTED: return "unsupported configuration";
+    case LBM_ERR_SEQUENCE: return "call out of sequence";
+    case LBM_ERR_CAPACITY: return "capacity exceeded";
+    case LBM_ERR_NOMEM: return "out of memory";
+    case LBM_ERR_CUDA: return "CUDA error";
+    case LBM_ERR_TIMEOUT: return "device wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int lbm_rope3d_tables(int head_dim, int ppf, int pph, int ppw, int patch_start_idx,
+                      double theta, lbm_rope_t** out) {
+  return lbm_rope3d_tables_fhw(head_dim, 0, 0, 0, ppf, pph, ppw, patch_start_idx, theta, 1.0,
+                               out);
+}
+
+int lbm_rope3d_tables_fhw(int head_dim, int dt, int dh, int dw, int ppf, int pph, int ppw,
+                          int patch_start_idx, double theta, double ntk_factor,
+                          lbm_rope_t** out) {
+  if (!out) return LBM_ERR_INVALID;
+  *out = nullptr;
+  if (head_dim < 6 || head_dim % 2) return LBM_ERR_INVALID;
+  if (dt == 0 && dh == 0 && dw == 0) {
+    // default split: d_h = d_w = 2 * (head_dim / 6), d_t = the rest; pairs ordered t, h, w
+    dh = dw = 2 * (head_dim / 6);
+    dt = head_dim - 2 * dh;
+  }
+  if (dt < 2 || dh < 2 || dw < 2 || dt % 2 || dh % 2 || dw % 2 || dt + dh + dw != head_dim ||
+      ppf < 1 || pph < 1 ||
+      ppw < 1 || patch_start_idx < 0 || !(ntk_factor > 0.0) || !(theta * ntk_factor > 1.0) ||
+      (long long)pph * ppw > (1 << 20) || ppf > (1 << 24))
+    return LBM_ERR_INVALID;
+  theta *= ntk_factor;  // [VideoRoPE] "NTK-Aware Frequency Scaling": theta * ntk_factor
+  lbm::RopeTables t{};
+  t.head_dim = head_dim;
+  t.ppf = ppf;
+  t.pph = pph;
+  t.ppw = ppw;
+  t.psi = patch_start_idx;
+  return build_rope(t, {ppf, dt, theta}, {pph + 1, dh, theta}, {ppw + 1, dw, theta}, out);
+}
+
+int lbm_rope2d_tables(int head_dim, int ppf, int pph, int ppw, int patch_start_idx,
+                      double frequency, lbm_rope_t** out) {
+  if (!out) return LBM_ERR_INVALID;
+  *out = nullptr;
+  // two halves (y, x) of whole feature pairs: head_dim divisible by 4
+  if (head_dim < 4 || head_dim % 4 || ppf < 1 || pph < 1 || ppw < 1 || patch_start_idx < 0 ||
+      !(frequency > 1.0) || (long long)pph * ppw > (1 << 20) || ppf > (1 << 24))
+    return LBM_ERR_INVALID;
+  lbm::RopeTables t{};
+  t.head_dim = head_dim;
+  t.ppf = ppf;
+  t.pph = pph;
+  t.ppw = ppw;
+  t.psi = patch_start_idx;
+  // [RoPERange] "Deriving Size from Token Count": each half's table has one row per token of
+  // a frame (positions 0 .. T-1), which covers the coordinates 0 .. max(pph, ppw) in use
+  const int rows = patch_start_idx + pph * ppw;
+  const int d_half = head_dim / 2;
+  return build_rope(t, {0, 0, frequency}, {rows, d_half, frequency}, {rows, d_half, frequency},
+                    out);
 }
 
 int lbm_rope3d_expand(const lbm_rope_t* rope, float* cos_out, float* sin_out, void* stream) {

@@ -10,12 +10,15 @@
 namespace lbm {
 
 // Per-axis cos/sin tables on the device, float2 (cos, sin), rounded once from double.
+// Feature pair i of a token at (t, h, w) takes the t table for i < nt, the h table for
+// nt <= i < nt + nh and the w table after.  The 2D (y, x) variant has nt = 0, its h and w
+// tables being the y and x halves (one row per token of a frame).
 struct RopeTables {
   int head_dim, ppf, pph, ppw, psi;
   int nt, nh, nw;          // pairs of the t, h, w axes (d_t/2, d_h/2, d_w/2)
-  const float2* tab_t;     // [ppf][nt]
-  const float2* tab_h;     // [pph + 1][nh]
-  const float2* tab_w;     // [ppw + 1][nw]
+  const float2* tab_t;     // [ppf][nt] (no rows when nt = 0)
+  const float2* tab_h;     // [pph + 1][nh] (2D: [psi + pph * ppw][nh])
+  const float2* tab_w;     // [ppw + 1][nw] (2D: [psi + pph * ppw][nw])
 };
 
 // Device pools of one cache.  Patch pools: [heads][num_pages * page_stride][head_dim];
@@ -72,10 +75,10 @@ struct AttnParams {
   int heads;
   int patches;           // valid tokens per patch page
   int page_stride;
-  int tiles_per_page;    // key tiles per patch page: ceil(patches / 128)
+  int tiles_per_page;    // key tiles per patch page: ceil(patches / attn_key_tile(D))
   int n_pages;           // visible patch pages
   int n_special;         // visible special tokens
-  int n_tiles;           // n_pages * tiles_per_page + ceil(n_special / 128)
+  int n_tiles;           // n_pages * tiles_per_page + ceil(n_special / attn_key_tile(D))
   int n_pairs;           // ceil(ceil(T / 128) / 2) query-tile pairs
   long long work;        // n_pairs * heads * n_tiles
   int grid;              // persistent CTAs

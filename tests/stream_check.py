@@ -65,9 +65,13 @@ def check_attn(got: np.ndarray, exact: np.ndarray, what: str) -> tuple[float, fl
 
 
 def make_cache(cfg: workloads.StreamConfig, max_frame_idx: int | None = None, split=None,
-               ntk_factor: float = 1.0):
+               ntk_factor: float = 1.0, rope2d_frequency: float | None = None):
     ppf = (max_frame_idx + 1) if max_frame_idx is not None else cfg.n_frames
-    rope = _lib.Rope3D(cfg.head_dim, ppf, cfg.pph, cfg.ppw, 6, split=split, ntk_factor=ntk_factor)
+    if rope2d_frequency is not None:
+        rope = _lib.Rope2D(cfg.head_dim, ppf, cfg.pph, cfg.ppw, 6, frequency=rope2d_frequency)
+    else:
+        rope = _lib.Rope3D(cfg.head_dim, ppf, cfg.pph, cfg.ppw, 6, split=split,
+                           ntk_factor=ntk_factor)
     cache = _lib.PagedKVCache(rope, cfg.heads, cfg.head_dim, cfg.patches, cfg.scale_frames,
                               cfg.sliding_window, max(1, cfg.n_keyframes),
                               _lib.LBM_BF16 if cfg.dtype == "bf16" else _lib.LBM_F32)
@@ -91,10 +95,12 @@ def regen_source(cfg: workloads.StreamConfig, frame_ids: list):
 
 def run_stream(cfg: workloads.StreamConfig, check_frames=None, rows=None, frame_ids=None,
                tamper=None, check_pools=True, regenerate=False, report=None, decide_after=False,
-               split=None, ntk_factor: float = 1.0, reset_at=()):
+               split=None, ntk_factor: float = 1.0, reset_at=(),
+               rope2d_frequency: float | None = None):
     """Streams every frame of cfg through the cache; checks the frames in check_frames.
 
     split, ntk_factor: RoPE variant (explicit (t, h, w) split, NTK factor), for both sides.
+    rope2d_frequency: rotate with the 2D (y, x) variant of that base frequency instead.
     reset_at: stream positions before which cache and oracle are reset (windowed streaming;
     frame_ids may then start again).
     decide_after: append every frame undecided and keep / drop it after its attention
@@ -108,11 +114,12 @@ def run_stream(cfg: workloads.StreamConfig, check_frames=None, rows=None, frame_
     import torch
     frame_ids = list(range(cfg.n_frames)) if frame_ids is None else list(frame_ids)
     check = set(range(cfg.n_frames)) if check_frames is None else set(check_frames)
-    rope, cache = make_cache(cfg, max(frame_ids), split, ntk_factor)
+    rope, cache = make_cache(cfg, max(frame_ids), split, ntk_factor, rope2d_frequency)
     so = ostream.StreamOracle(cfg.heads, cfg.head_dim, cfg.pph, cfg.ppw, cfg.scale_frames,
                               cfg.sliding_window, max(1, cfg.n_keyframes),
                               kv_source=regen_source(cfg, frame_ids) if regenerate else None,
-                              split=split, ntk_factor=ntk_factor)
+                              split=split, ntk_factor=ntk_factor,
+                              rope2d_frequency=rope2d_frequency)
     summary = []
     T = cfg.tokens
     keys = cfg.keyframes

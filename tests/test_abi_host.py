@@ -172,13 +172,20 @@ def test_pager_decision_after_attention_errors(lib):
 
 def test_rope_variant_argument_checks_without_gpu(lib):
     h = ctypes.c_void_p()
-    for args in [(20, 22, 21), (0, 32, 32), (21, 21, 22)]:          # odd or empty axes
+    for args in [(64, 20, 22, 21), (64, 0, 32, 32), (64, 21, 21, 22),   # odd or empty axes
+                 (64, 20, 22, 24), (4, 0, 0, 0), (63, 0, 0, 0)]:       # wrong sum, bad head_dim
         assert lib.lbm_rope3d_tables_fhw(*args, 4, 3, 3, 6, 10000.0, 1.0,
                                          ctypes.byref(h)) == _lib.LBM_ERR_INVALID
-    assert lib.lbm_rope3d_tables_fhw(20, 22, 22, 4, 3, 3, 6, 10000.0, 0.0,
+    assert lib.lbm_rope3d_tables_fhw(64, 20, 22, 22, 4, 3, 3, 6, 10000.0, 0.0,
                                      ctypes.byref(h)) == _lib.LBM_ERR_INVALID   # ntk <= 0
-    assert lib.lbm_rope3d_tables_fhw(20, 22, 22, 4, 3, 3, 6, 1.0, 0.5,
+    assert lib.lbm_rope3d_tables_fhw(64, 20, 22, 22, 4, 3, 3, 6, 1.0, 0.5,
                                      ctypes.byref(h)) == _lib.LBM_ERR_INVALID   # theta*ntk <= 1
+    assert lib.lbm_rope3d_tables_fhw(64, 0, 0, 0, 4, 3, 3, 6, 1.0, 0.5,
+                                     ctypes.byref(h)) == _lib.LBM_ERR_INVALID   # default split too
+    # the 2D variant: head_dim a multiple of 4, frequency > 1
+    for hd, freq in [(66, 100.0), (2, 100.0), (64, 1.0), (64, 0.0)]:
+        assert lib.lbm_rope2d_tables(hd, 4, 3, 3, 6, freq, ctypes.byref(h)) == _lib.LBM_ERR_INVALID
+    assert lib.lbm_rope2d_tables(64, 4, 3, 3, 6, 100.0, None) == _lib.LBM_ERR_INVALID
 
 
 def test_create_argument_checks_without_gpu(lib):

@@ -70,6 +70,43 @@ def test_rope_variant_stream(head_dim, split, ntk):
                split=split, ntk_factor=ntk)
 
 
+@pytest.mark.parametrize("head_dim,ppf,pph,ppw", [(64, 4, 9, 11), (128, 3, 64, 64)])
+def test_rope2d_tables_match_oracle(head_dim, ppf, pph, ppw):
+    """The 2D (y, x) variant ("How to Handle Sequences Exceeding the RoPE Training Range in
+    LingBot-Map"): the tables the library builds, expanded per token, equal the oracle's."""
+    import torch
+    from oracle import rope2d
+    rope = _lib.Rope2D(head_dim, ppf, pph, ppw, 6, frequency=100.0)
+    rows = ppf * (6 + pph * ppw)
+    cos = torch.empty(rows, head_dim // 2, device="cuda")
+    sin = torch.empty_like(cos)
+    rope.expand(cos, sin)
+    torch.cuda.synchronize()
+    ec, es = rope2d.expanded_table(head_dim, ppf, pph, ppw, 6, 100.0)
+    assert np.abs(cos.cpu().numpy() - ec).max() <= 1e-5
+    assert np.abs(sin.cpu().numpy() - es).max() <= 1e-5
+    rope.close()
+
+
+@pytest.mark.parametrize("head_dim", [64, 128])
+def test_rope2d_stream_all_frames_all_rows(head_dim):
+    """Fused rotate + append and attention with the 2D variant: q, pages, page table and
+    outputs match the oracle rotating by (y, x) with base frequency 100."""
+    run_stream(custom_config(222 + head_dim // 64, 2, head_dim, "bf16", 7, 9, 8, 2, 1, 2),
+               rope2d_frequency=100.0)
+
+
+def test_rope2d_64x64_grid_sampled():
+    """The page's high-resolution case: a 64 x 64 grid (4096 patch tokens), 8 heads x 128;
+    135 sampled query rows (all specials, the last row, 128 random) at every frame."""
+    cfg = custom_config(225, 8, 128, "bf16", 64, 64, 5, 1, 1, 2, v_dist="uniform")
+    rng = np.random.default_rng(225)
+    rows = np.unique(np.concatenate([np.arange(6), [cfg.tokens - 1],
+                                     rng.choice(np.arange(6, cfg.tokens - 1), 128,
+                                                replace=False)]))
+    run_stream(cfg, rows=rows, rope2d_frequency=100.0)
+
+
 def test_tiny_fp32_config_all_frames():
     run_stream(CONFIGS[0])
 
@@ -158,7 +195,9 @@ def test_full_size_config_sampled(cid, frames):
     cfg = CONFIGS[cid]
     rng = np.random.default_rng(cid)
     rows = np.unique(np.concatenate([np.arange(6), [cfg.tokens - 1],
-                                     rng.choice(cfg.tokens, 120, replace=False)]))
+                                     rng.choice(np.arange(6, cfg.tokens - 1), 128,
+                                                replace=False)]))
+    assert len(rows) == 128 + 7
     run_stream(cfg, check_frames=frames, rows=rows, regenerate=True)
 
 
@@ -166,10 +205,14 @@ def test_full_size_config_sampled(cid, frames):
 def test_long_stream_2000_keyframes_sampled():
     cfg = CONFIGS[3]
     rng = np.random.default_rng(3)
+    # every special row, the last row and 128 random rows (>= 128 query rows, all heads);
+    # pools (K rotated at t up to 1999, V copied) checked at every sampled frame
     rows = np.unique(np.concatenate([np.arange(6), [cfg.tokens - 1],
-                                     rng.choice(cfg.tokens, 58, replace=False)]))
+                                     rng.choice(np.arange(6, cfg.tokens - 1), 128,
+                                                replace=False)]))
+    assert len(rows) >= 128 + 7
     run_stream(cfg, check_frames=[0, 135, 136, 137, 1000, 1999], rows=rows, regenerate=True,
-               check_pools=False)
+               check_pools=True)
 
 
 @pytest.mark.parametrize("head_dim", [64, 128])
