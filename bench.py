@@ -5,13 +5,19 @@
 One step streams every frame of the workload through a fresh cache: per frame one
 lbm_append_frame (fused rotate + append) and one lbm_attend_frame (paged attention on
 persistent CTAs, plus the combine of the units several CTAs share), host page-table
-bookkeeping included.  The default workload is the 768-patch stream: 16 heads x head_dim 64, bf16,
-6 special + 24x32 patch tokens per frame, 64 keyframes, scale_frames 8, sliding_window 16.
-Inputs are seeded synthetic frames; the 64 frames of a step (304 MB of q/k/v) are larger
-than L2, so no input is L2-resident between steps.
+bookkeeping included.  The default workload is the 4096-patch stream (configuration 4):
+8 heads x head_dim 128, bf16, 6 special + 64x64 patch tokens per frame, 96 keyframes,
+scale_frames 4, sliding_window 32.  Inputs are seeded synthetic frames held in HBM before
+timing; a pool of up to 64 distinct frames (1.6 GB here) is larger than L2, so no input is
+L2-resident when a frame reads it.
 
-With N > 1 (torchrun) every rank streams its own independent copy of the workload (the step
-has no exchange between GPUs): weak scaling, value = all ranks' frames / max rank time.
+The same invocation (N = 1) also measures the 999-patch streams (configurations 2 and 3:
+keyframe every 5th frame over 320 frames, and 2000 keyframes) and reports their attention
+and append roofline fractions under "other_configs", each with its own clock summary.
+
+With N > 1 (torchrun) every rank streams its own independent copy of the headline workload
+(the step has no exchange between GPUs): weak scaling, value = all ranks' frames / max rank
+time.
 
 Prints one JSON line (rank 0).  ``--impl reference`` times the fp64 CPU oracle on this
 host's cores on a bounded sample of the same workload instead.
@@ -34,8 +40,12 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 INPUT_POOL = 64
+HEADLINE_CONFIG = 4
+OTHER_CONFIGS = (2, 3)
 METRIC = "streamed frames/s per layer (RoPE+append+paged attn); % of bf16 TC / HBM peak"
 UNIT = "frames/s"
+# ncu summaries whose DRAM bytes per attention launch give roofline.traffic (per config)
+TRAFFIC_PROFILES = {4: "attn_tc_large4096.md", 1: "attn_tc_stream768.md"}
 
 
 def _peaks():
@@ -50,12 +60,25 @@ def _peaks():
             "source": "fallback"}
 
 
-def measured_traffic(avg_keys: float):
-    """DRAM bytes per attention launch from the committed ncu summary, scaled from the
-    captured frame's key count to the stream's average (K/V reads dominate and grow with
-    the keys); None once the kernel source differs from the one that was profiled."""
+def tensor_peak(peaks: dict, clocks: dict) -> tuple[float, str]:
+    """The bf16 peak the attention is compared with: the sustained (power-capped) figure when
+    the clocks sampled during the timed region show the power cap, else the burst figure."""
+    if "sw_power_cap" in (clocks.get("reasons") or []):
+        return peaks["bf16_tflops_sustained"], (peaks["source"] + " bf16_tflops_sustained "
+                                                "(sw_power_cap seen during the timed region)")
+    return peaks["bf16_tflops"], peaks["source"] + " bf16_tflops (burst; no power cap seen)"
+
+
+def measured_traffic(cid: int, avg_keys: float):
+    """DRAM bytes per attention launch from the committed ncu summary of this workload,
+    scaled from the captured frame's key count to the stream's average (K/V reads dominate
+    and grow with the keys); None when there is no summary or the kernel source differs from
+    the one that was profiled."""
     import hashlib
-    prof = os.path.join(ROOT, "profiles", "attn_tc_stream768.md")
+    name = TRAFFIC_PROFILES.get(cid)
+    if name is None:
+        return None
+    prof = os.path.join(ROOT, "profiles", name)
     src = os.path.join(ROOT, "rope_paged_kv_02_b200", "csrc", "attn_tc.cu")
     if not os.path.exists(prof):
         return None
@@ -74,7 +97,7 @@ def measured_traffic(avg_keys: float):
         return None
 
 
-def frame_work(cfg):
+def frame_work(cfg, n_frames: int | None = None):
     """Algorithmic work per frame of a stream: (attention FLOPs, append bytes, keys seen).
 
     Frame n with m keyframes committed before it sees min(m, S+W)+1 patch pages and 6(m+1)
@@ -84,7 +107,7 @@ def frame_work(cfg):
     T, H, D, e = cfg.tokens, cfg.heads, cfg.head_dim, cfg.elem_bytes
     flops, nbytes, keys = [], [], []
     m = 0
-    for key in cfg.keyframes:
+    for key in cfg.keyframes[:n_frames]:
         nk = (min(m, cfg.scale_frames + cfg.sliding_window) + 1) * cfg.patches + 6 * (m + 1)
         flops.append(4.0 * T * nk * H * D)
         nbytes.append(6.0 * T * H * D * e)
@@ -185,60 +208,9 @@ def barrier(world: int):
         dist.barrier()
 
 
-def run_reference(args, cfg, rank, world):
-    """The fp64 oracle on this host's cores, bounded sample of the same workload."""
-    if rank != 0:
-        return None
-    from oracle import stream as ostream
-    from rope_paged_kv_02_b200 import workloads
-    sample_frames = [cfg.scale_frames + cfg.sliding_window + 1]  # a steady-state frame
-    so_frames = sample_frames[-1] + 1
-
-    def one_step():
-        so = ostream.StreamOracle(cfg.heads, cfg.head_dim, cfg.pph, cfg.ppw, cfg.scale_frames,
-                                  cfg.sliding_window, cfg.n_keyframes,
-                                  kv_source=_regen(cfg))
-        t_att = 0.0
-        for f in range(so_frames):
-            q, k, v = workloads.frame_qkv(cfg, f)
-            t0 = time.perf_counter()
-            so.step(f, cfg.keyframes[f], q, k, v, rows=None if f in sample_frames else [],
-                    attend=f in sample_frames)
-            if f in sample_frames:
-                t_att += time.perf_counter() - t0
-        return t_att / len(sample_frames)
-
-    for _ in range(args.warmup):
-        one_step()
-    times = [one_step() for _ in range(args.steps)]
-    per_frame = float(np.mean(times))
-    value = 1.0 / per_frame
-    cores = _blas_threads()
-    line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
-        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": per_frame * 1e3, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, bf16-valued inputs)",
-        "config": _config_dict(cfg, world),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": f"one steady-state frame ({sample_frames[0]}) of the stream "
-                                   f"per step, all {cfg.tokens} query rows x {cfg.heads} heads, "
-                                   "rotate + page state + attention in fp64"},
-        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-    }
-    return line
-
-
-def _regen(cfg):
-    from rope_paged_kv_02_b200 import workloads
-
-    def source(frame, region):
-        if region == "special":
-            return workloads.frame_specials(cfg, frame, 1), workloads.frame_specials(cfg, frame, 2)
-        return workloads.frame_tensor(cfg, frame, 1)[6:], workloads.frame_tensor(cfg, frame, 2)[6:]
-
-    return source
-
+# ------------------------------------------------------------------------------------------
+# the fp64 oracle on the host cores (reference arm and cpu_baseline)
+# ------------------------------------------------------------------------------------------
 
 def _blas_threads() -> int:
     try:
@@ -251,192 +223,246 @@ def _blas_threads() -> int:
     return os.cpu_count() or 1
 
 
-def _config_dict(cfg, world):
-    return {"workload": cfg.describe(), "frames_per_step": cfg.n_frames,
-            "tokens_per_frame": cfg.tokens, "heads": cfg.heads, "head_dim": cfg.head_dim,
-            "scale_frames": cfg.scale_frames, "sliding_window": cfg.sliding_window,
-            "parallelism": f"replicas x{world} (independent streams, no exchange)",
-            "l2": "inputs larger than L2 (%d distinct frames of q/k/v cycled, %.0f MB)" % (
-                min(cfg.n_frames, INPUT_POOL),
-                min(cfg.n_frames, INPUT_POOL) * 3 * cfg.tokens * cfg.heads * cfg.head_dim
-                * cfg.elem_bytes / 1e6)}
+def _busiest_frame(cfg) -> int:
+    """First frame that sees the stream's largest number of patch pages (steady state)."""
+    m, best, first = 0, -1, 0
+    for f, key in enumerate(cfg.keyframes):
+        n_pages = min(m, cfg.scale_frames + cfg.sliding_window) + 1
+        if n_pages > best:
+            best, first = n_pages, f
+        if key:
+            m += 1
+    return first
+
+
+class OracleSampler:
+    """The fp64 oracle (``oracle.stream.StreamOracle``, as it stands) advanced to the busiest
+    frame of the stream, then timed on frames that see that frame's retained keys.
+
+    Query rows are independent, so a frame's attention is timed on a sample of rows: each
+    sample steps the oracle over one frame twice, with r1 and then r2 sampled rows (the frame
+    index increases and the frames are stepped as non-keyframes, so the retained set and the
+    key count stay those of the busiest frame).  Per-frame time = t(r1) + (T - r1) * slope,
+    slope = (t(r2) - t(r1)) / (r2 - r1): rotation, page-table work and key gathering are
+    counted once, the attention once per row."""
+
+    def __init__(self, cfg):
+        from oracle import stream as ostream
+        from rope_paged_kv_02_b200 import workloads
+        self.cfg = cfg
+        self.wl = workloads
+        self.so = ostream.StreamOracle(cfg.heads, cfg.head_dim, cfg.pph, cfg.ppw,
+                                       cfg.scale_frames, cfg.sliding_window,
+                                       max(1, cfg.n_keyframes))
+        self.frame = _busiest_frame(cfg)
+        for f in range(self.frame):            # untimed: build the retained state
+            q, k, v = workloads.frame_qkv(cfg, f)
+            self.so.step(f, cfg.keyframes[f], q, k, v, rows=[], attend=False)
+        self.next = self.frame
+        self.r2 = min(64, cfg.tokens)
+        self.r1 = max(1, self.r2 // 2)
+        self.rng = np.random.default_rng(12345)
+
+    def _timed(self, n_rows: int) -> float:
+        q, k, v = self.wl.frame_qkv(self.cfg, self.next)
+        rows = np.sort(self.rng.choice(self.cfg.tokens, n_rows, replace=False))
+        t0 = time.perf_counter()
+        self.so.step(self.next, False, q, k, v, rows=rows, attend=True)
+        dt = time.perf_counter() - t0
+        self.next += 1
+        return dt
+
+    def frame_seconds(self) -> tuple[float, float]:
+        """(estimated seconds per full frame, seconds spent)."""
+        t1 = self._timed(self.r1)
+        t2 = self._timed(self.r2)
+        slope = max(t2 - t1, 0.0) / (self.r2 - self.r1)
+        return t1 + (self.cfg.tokens - self.r1) * slope, t1 + t2
+
+    def describe(self) -> str:
+        c = self.cfg
+        return (f"frames >= {self.frame} (the first to see as many patch pages as the "
+                f"stream ever does), stepped as "
+                f"non-keyframes so each sees the same keys; {self.r1} and {self.r2} random "
+                f"query rows x {c.heads} heads per sample, full fp64 step (rotate q/k, page "
+                f"state, attention), per-frame time extrapolated linearly in rows to all "
+                f"{c.tokens}")
+
+
+def run_reference(args, cfg, rank, world):
+    """The fp64 oracle on this host's cores, bounded sample of the same workload."""
+    if rank != 0:
+        return None
+    sampler = OracleSampler(cfg)
+    for _ in range(args.warmup):
+        sampler.frame_seconds()
+    times = [sampler.frame_seconds()[0] for _ in range(args.steps)]
+    per_frame = float(np.mean(times))
+    value = 1.0 / per_frame
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": per_frame * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, bf16-valued inputs)",
+        "config": _config_dict(cfg, world),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": _blas_threads(),
+                         "kind": "oracle",
+                         "sample": "one frame per step: " + sampler.describe()},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    return line
 
 
 def cpu_baseline(cfg):
-    """Oracle frames/s on a bounded sample (two steady-state frames, all rows)."""
-    from oracle import stream as ostream
-    from rope_paged_kv_02_b200 import workloads
-    targets = [cfg.scale_frames + cfg.sliding_window + 1, cfg.scale_frames + cfg.sliding_window + 2]
-    so = ostream.StreamOracle(cfg.heads, cfg.head_dim, cfg.pph, cfg.ppw, cfg.scale_frames,
-                              cfg.sliding_window, cfg.n_keyframes, kv_source=_regen(cfg))
-    spent = 0.0
-    for f in range(targets[-1] + 1):
-        q, k, v = workloads.frame_qkv(cfg, f)
-        t0 = time.perf_counter()
-        so.step(f, cfg.keyframes[f], q, k, v, rows=None if f in targets else [],
-                attend=f in targets)
-        if f in targets:
-            spent += time.perf_counter() - t0
-    return {"value": len(targets) / spent, "unit": UNIT, "cores": _blas_threads(),
+    """Oracle frames/s on a bounded sample (two frames' worth of row samples)."""
+    sampler = OracleSampler(cfg)
+    est, spent = [], 0.0
+    for _ in range(2):
+        e, s = sampler.frame_seconds()
+        est.append(e)
+        spent += s
+    return {"value": 1.0 / float(np.mean(est)), "unit": UNIT, "cores": _blas_threads(),
             "kind": "oracle",
-            "sample": f"frames {targets} of the stream (steady state), all {cfg.tokens} rows "
-                      f"x {cfg.heads} heads, fp64 rotate + page state + attention; "
-                      f"{spent:.1f} s of CPU work"}
+            "sample": "two samples: " + sampler.describe() + f"; {spent:.1f} s of CPU work"}
 
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--config", type=int, default=1)
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    args = ap.parse_args()
-
-    rank, world, local = dist_setup(args.gpus)
-    from rope_paged_kv_02_b200 import workloads
-    cfg = workloads.CONFIGS[args.config]
-
-    if args.impl == "reference":
-        line = run_reference(args, cfg, rank, world)
-        if line is not None:
-            print(json.dumps(line), flush=True)
-        _teardown(world)
-        return
-
-    import torch
-    from rope_paged_kv_02_b200 import _lib
-    from rope_paged_kv_02_b200.build import build
-    if rank == 0 or not os.path.exists(_lib.LIB_PATH):
-        build()
-    barrier(world)
-    _lib.load()
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    tdt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
-
-    # ---- inputs resident in HBM before timing: the frames of the stream, or for streams
-    # longer than INPUT_POOL frames a pool of that many distinct frames used in turn (the
-    # pool is larger than L2, and the cache's contents do not change the work per frame) ----
-    F = cfg.n_frames
+def _config_dict(cfg, world, n_frames=None):
+    F = cfg.n_frames if n_frames is None else n_frames
     pool = min(F, INPUT_POOL)
-    qs, ks, vs = [], [], []
-    for f in range(pool):
-        q, k, v = workloads.frame_qkv(cfg, f)
-        qs.append(torch.from_numpy(q).to(dev, tdt))
-        ks.append(torch.from_numpy(k).to(dev, tdt))
-        vs.append(torch.from_numpy(v).to(dev, tdt))
-    outs = [torch.empty_like(qs[0]) for _ in range(pool)]
-    rope = _lib.Rope3D(cfg.head_dim, F, cfg.pph, cfg.ppw, 6)
-    cache = _lib.PagedKVCache(rope, cfg.heads, cfg.head_dim, cfg.patches, cfg.scale_frames,
-                              cfg.sliding_window, cfg.n_keyframes,
-                              _lib.LBM_BF16 if cfg.dtype == "bf16" else _lib.LBM_F32)
-    stream = torch.cuda.current_stream(dev)
-    keys = cfg.keyframes
+    d = {"workload": cfg.describe() if n_frames is None else
+         f"first {n_frames} frames of " + cfg.describe(),
+         "frames_per_step": F,
+         "tokens_per_frame": cfg.tokens, "heads": cfg.heads, "head_dim": cfg.head_dim,
+         "scale_frames": cfg.scale_frames, "sliding_window": cfg.sliding_window,
+         "parallelism": f"replicas x{world} (independent streams, no exchange)",
+         "l2": "inputs larger than L2 (%d distinct frames of q/k/v cycled, %.0f MB)" % (
+             pool, pool * 3 * cfg.tokens * cfg.heads * cfg.head_dim * cfg.elem_bytes / 1e6)}
+    return d
 
-    def step(ev=None):
-        cache.reset()
-        for f in range(F):
-            b = f % pool
+
+# ------------------------------------------------------------------------------------------
+# the CUDA path
+# ------------------------------------------------------------------------------------------
+
+class Workload:
+    """Device (and pinned host) copies of a stream's input pool, a cache, and the step."""
+
+    def __init__(self, cfg, dev, n_frames=None, host_copies=False):
+        import torch
+        from rope_paged_kv_02_b200 import _lib, workloads
+        self.cfg = cfg
+        self.F = cfg.n_frames if n_frames is None else n_frames
+        self.pool = min(self.F, INPUT_POOL)
+        tdt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+        self.tdt = tdt
+        self.q, self.k, self.v, self.host = [], [], [], []
+        for f in range(self.pool):
+            ts = [torch.from_numpy(x).to(tdt) for x in workloads.frame_qkv(cfg, f)]
+            if host_copies:
+                ts = [t.pin_memory() for t in ts]
+                self.host.append(ts)
+            self.q.append(ts[0].to(dev))
+            self.k.append(ts[1].to(dev))
+            self.v.append(ts[2].to(dev))
+        self.out = [torch.empty_like(self.q[0]) for _ in range(self.pool)]
+        self.rope = _lib.Rope3D(cfg.head_dim, max(self.F, cfg.n_frames), cfg.pph, cfg.ppw, 6)
+        self.cache = _lib.PagedKVCache(self.rope, cfg.heads, cfg.head_dim, cfg.patches,
+                                       cfg.scale_frames, cfg.sliding_window,
+                                       max(1, cfg.n_keyframes),
+                                       _lib.LBM_BF16 if cfg.dtype == "bf16" else _lib.LBM_F32)
+        self.keys = cfg.keyframes
+
+    def step(self, stream, ev=None):
+        """One pass over the stream; with ev, an event pair around every append and attend."""
+        c = self.cache
+        c.reset()
+        for f in range(self.F):
+            b = f % self.pool
             if ev is not None:
                 ev[f][0].record(stream)
-            cache.append_frame(qs[b], ks[b], vs[b], f, keys[f], stream)
+            c.append_frame(self.q[b], self.k[b], self.v[b], f, self.keys[f], stream)
             if ev is not None:
                 ev[f][1].record(stream)
-            cache.attend_frame(qs[b], outs[b], stream)
+            c.attend_frame(self.q[b], self.out[b], stream)
             if ev is not None:
                 ev[f][2].record(stream)
 
-    for _ in range(max(3, args.warmup)):
-        step()
+    def close(self):
+        self.cache.close()
+        self.rope.close()
+
+
+def measure(w: Workload, steps: int, warmup: int, world: int, local: int, peaks: dict,
+            dev) -> dict:
+    """Times `steps` steps of the stream (after `warmup`), then a second pass of the same
+    steps with an event pair around every kernel launch; returns the figures of one line."""
+    import torch
+    cfg = w.cfg
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(warmup):
+        w.step(stream)
     torch.cuda.synchronize()
-    cache.check()
+    w.cache.check()
 
     # ---- timed region: K steps back to back on the stream, bracketed by two events ----
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    launches0 = cache.state()["kernel_launches"]
+    launches0 = w.cache.state()["kernel_launches"]
     with ClockSampler(local) as clocks:
         barrier(world)
         torch.cuda.synchronize()
         t0.record(stream)
-        for s in range(args.steps):
-            step()
+        for _ in range(steps):
+            w.step(stream)
         t1.record(stream)
         torch.cuda.synchronize()
         barrier(world)
-    launches = cache.state()["kernel_launches"] - launches0
-    ms = t0.elapsed_time(t1)
-    ms_max = max_over_ranks(ms, world)
-    cache.check()
+    launches = w.cache.state()["kernel_launches"] - launches0
+    ms = max_over_ranks(t0.elapsed_time(t1), world)
+    w.cache.check()
 
     # ---- per-kernel durations: the same K steps again with an event pair around every
-    # append and every attend launch on the launching stream.  The events between launches
-    # stop each kernel from overlapping its predecessor's tail (programmatic dependent
-    # launch), so these durations are slightly pessimistic; the headline uses the pass above.
-    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(F)]
-           for _ in range(args.steps)]
+    # append and every attend launch (attention + combine) on the launching stream ----
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(w.F)]
+           for _ in range(steps)]
     barrier(world)
     torch.cuda.synchronize()
-    for s in range(args.steps):
-        step(evs[s])
+    for s in range(steps):
+        w.step(stream, evs[s])
     torch.cuda.synchronize()
     barrier(world)
-    cache.check()
+    w.cache.check()
     append_ms = np.array([[e[0].elapsed_time(e[1]) for e in st] for st in evs])
     attn_ms = np.array([[e[1].elapsed_time(e[2]) for e in st] for st in evs])
 
-    flops, nbytes, keys = frame_work(cfg)
-    frames_total = F * args.steps * world
-    value = frames_total / (ms_max / 1e3)
-    peaks = _peaks()
-    attn_avg_s = attn_ms.mean() / 1e3
-    attn_tflops = flops.mean() / attn_avg_s / 1e12
-    append_gbs = nbytes.mean() / (append_ms.mean() / 1e3) / 1e9
-    # steady-state frames (window full) for the headline roofline of the attention kernel
-    ss = slice(cfg.scale_frames + cfg.sliding_window, F)
-    ss_tflops = flops[ss].mean() / (attn_ms[:, ss].mean() / 1e3) / 1e12
-
-    # ---- end to end: host (pinned) inputs -> device -> append/attend -> host output ----
-    e2e = e2e_measure(cfg, cache, args, dev, tdt, world)
-
-    line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_max / args.steps,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype,
-        "data": "synthetic (seeded N(0,1) q/k/v rounded to bf16)",
-        "config": _config_dict(cfg, world),
-        "roofline": {
-            "bound": "tensor", "achieved": attn_tflops,
-            "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-            "frac": attn_tflops / peaks["bf16_tflops_sustained"],
-            "traffic": measured_traffic(float(keys.mean())) if args.config == 1 else None,
-            "kernel": "paged attention (attn_tc + stream-K combine), all frames",
-            "kernel_timing": "event pair around every attend launch, second pass of the "
-                             "same K steps",
-            "peak_source": peaks["source"] + " bf16_tflops_sustained",
-            "steady_state_achieved": ss_tflops,
-        },
+    flops, nbytes, keys = frame_work(cfg, w.F)
+    step_ms = ms / steps
+    # The events between launches stop a kernel from overlapping its predecessor's tail, so
+    # the event-pair sums can exceed the undisturbed step.  The attention time used for the
+    # roofline is capped so that attention + append never exceed the timed step.
+    attn_step_evt = float(attn_ms.sum(axis=1).mean())
+    append_step_evt = float(append_ms.sum(axis=1).mean())
+    attn_step = min(attn_step_evt, step_ms - append_step_evt)
+    clk = clocks.summary()
+    peak, peak_src = tensor_peak(peaks, clk)
+    attn_tflops = flops.sum() / (attn_step / 1e3) / 1e12
+    append_gbs = nbytes.sum() / (append_step_evt / 1e3) / 1e9
+    return {
+        "frames_per_s": w.F * steps * world / (ms / 1e3), "ms_per_step": step_ms,
+        "steps": steps, "warmup": warmup, "gpu_launches": int(launches),
+        "attention": {
+            "achieved_tflops": attn_tflops, "peak_tflops": peak, "frac": attn_tflops / peak,
+            "peak_source": peak_src, "ms_per_step": attn_step,
+            "event_pair_ms_per_step": attn_step_evt,
+            "avg_us": attn_step / w.F * 1e3, "flops_per_frame_avg": float(flops.mean()),
+            "avg_keys": float(keys.mean())},
         "append": {"achieved_gbs": append_gbs, "peak_gbs": peaks["hbm_gbs"],
                    "frac": append_gbs / peaks["hbm_gbs"], "bytes_per_frame": float(nbytes[0]),
-                   "avg_us": float(append_ms.mean() * 1e3)},
-        "attention": {"avg_us": float(attn_ms.mean() * 1e3),
-                      "steady_state_avg_us": float(attn_ms[:, ss].mean() * 1e3),
-                      "flops_per_frame_avg": float(flops.mean())},
-        "e2e": e2e,
-        "gpu_launches": int(launches),
-        "clocks": clocks.summary(),
+                   "avg_us": append_step_evt / w.F * 1e3},
+        "clocks": clk,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(cfg)
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-    cache.close()
-    rope.close()
-    _teardown(world)
 
 
-def e2e_measure(cfg, cache, args, dev, tdt, world):
+def e2e_measure(w: Workload, steps: int, world: int, dev):
     """Same metric through the C ABI with host buffers: per frame, pinned host q/k/v are
     copied to the device on a host-to-device stream, the frame is appended and attended on
     the compute stream, and its output is copied back to pinned host memory on a
@@ -444,16 +470,11 @@ def e2e_measure(cfg, cache, args, dev, tdt, world):
     buffer sets rotate: a frame's inputs are overwritten only after the frame that last used
     them has been attended, its output only after the previous one has been copied out."""
     import torch
-    F = cfg.n_frames
-    from rope_paged_kv_02_b200 import workloads
-    hq, hk, hv, ho = [], [], [], []
-    pool = min(F, INPUT_POOL)
-    for f in range(pool):
-        q, k, v = workloads.frame_qkv(cfg, f)
-        hq.append(torch.from_numpy(q).to(tdt).pin_memory())
-        hk.append(torch.from_numpy(k).to(tdt).pin_memory())
-        hv.append(torch.from_numpy(v).to(tdt).pin_memory())
-        ho.append(torch.empty_like(hq[-1]).pin_memory())
+    F, pool, tdt, cache = w.F, w.pool, w.tdt, w.cache
+    hq = [h[0] for h in w.host]
+    hk = [h[1] for h in w.host]
+    hv = [h[2] for h in w.host]
+    ho = [torch.empty_like(hq[0]).pin_memory() for _ in range(pool)]
     nbuf = 3
     dq = [torch.empty(hq[0].shape, dtype=tdt, device=dev) for _ in range(nbuf)]
     dk = [torch.empty_like(dq[0]) for _ in range(nbuf)]
@@ -465,7 +486,7 @@ def e2e_measure(cfg, cache, args, dev, tdt, world):
     attended = [torch.cuda.Event() for _ in range(nbuf)]  # the frame in buffer b attended
     landed = [torch.cuda.Event() for _ in range(nbuf)]    # inputs of buffer b on the device
     copied = [torch.cuda.Event() for _ in range(nbuf)]    # output of buffer b on the host
-    keys = cfg.keyframes
+    keys = w.keys
 
     def step(first):
         cache.reset()
@@ -498,15 +519,106 @@ def e2e_measure(cfg, cache, args, dev, tdt, world):
     barrier(world)
     torch.cuda.synchronize()
     t0.record(comp)
-    for _ in range(args.steps):
+    for _ in range(steps):
         step(False)
     comp.wait_stream(d2h)          # the last outputs are on the host
     t1.record(comp)
     torch.cuda.synchronize()
     ms = max_over_ranks(t0.elapsed_time(t1), world)
     per = hq[0].numel() * hq[0].element_size()
-    return {"value": F * args.steps * world / (ms / 1e3), "unit": UNIT,
+    return {"value": F * steps * world / (ms / 1e3), "unit": UNIT,
             "h2d_bytes_per_step": 3 * per * F, "d2h_bytes_per_step": per * F}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", type=int, default=HEADLINE_CONFIG)
+    ap.add_argument("--frames", type=int, default=None,
+                    help="stream only the first N frames (small profiling cases)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-other-configs", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+
+    rank, world, local = dist_setup(args.gpus)
+    from rope_paged_kv_02_b200 import workloads
+    cfg = workloads.CONFIGS[args.config]
+
+    if args.impl == "reference":
+        line = run_reference(args, cfg, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        _teardown(world)
+        return
+
+    import torch
+    from rope_paged_kv_02_b200 import _lib
+    from rope_paged_kv_02_b200.build import build
+    if rank == 0 or not os.path.exists(_lib.LIB_PATH):
+        build()
+    barrier(world)
+    _lib.load()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks = _peaks()
+    warmup = max(3, args.warmup)
+
+    w = Workload(cfg, dev, args.frames, host_copies=not args.no_e2e)
+    head = measure(w, args.steps, warmup, world, local, peaks, dev)
+    e2e = None if args.no_e2e else e2e_measure(w, args.steps, world, dev)
+    _, _, keys = frame_work(cfg, w.F)
+    w.close()
+    del w
+    torch.cuda.empty_cache()
+
+    att, app = head["attention"], head["append"]
+    line = {
+        "metric": METRIC, "value": head["frames_per_s"], "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": warmup, "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype,
+        "data": "synthetic (seeded q/k/v rounded to bf16)",
+        "config": _config_dict(cfg, world, args.frames),
+        "roofline": {
+            "bound": "tensor", "achieved": att["achieved_tflops"], "peak": att["peak_tflops"],
+            "unit": "TFLOP/s", "frac": att["frac"],
+            "traffic": measured_traffic(args.config, float(keys.mean())),
+            "kernel": "paged attention (attn_tc + stream-K combine), all frames of the stream",
+            "kernel_timing": "event pair around every attend launch in a second pass of the "
+                             "same K steps; per-step sum capped at ms_per_step minus the "
+                             "appends' event-pair time",
+            "peak_source": att["peak_source"],
+        },
+        "append": app,
+        "attention": att,
+        "e2e": e2e,
+        "gpu_launches": head["gpu_launches"],
+        "clocks": head["clocks"],
+    }
+    if world == 1 and not args.no_other_configs and args.frames is None:
+        others = {}
+        for cid in OTHER_CONFIGS:
+            if cid == args.config:
+                continue
+            ocfg = workloads.CONFIGS[cid]
+            ow = Workload(ocfg, dev)
+            # the 2000-frame stream takes ~2 s a step: two timed steps bound its time
+            osteps = 2 if ocfg.n_frames > 1000 else min(args.steps, 5)
+            r = measure(ow, osteps, 3, world, local, peaks, dev)
+            ow.close()
+            del ow
+            torch.cuda.empty_cache()
+            r["workload"] = ocfg.describe()
+            others[ocfg.name] = r
+        line["other_configs"] = others
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    _teardown(world)
 
 
 def _teardown(world):
