@@ -3,9 +3,11 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config C]
 
 One step streams every frame of the workload through a fresh cache: per frame one
-lbm_append_frame (fused rotate + append) and one lbm_attend_frame (paged attention on
-persistent CTAs, plus the combine of the units several CTAs share), host page-table
-bookkeeping included.  The default workload is the 4096-patch stream (configuration 4):
+lbm_append_frame (fused rotate + append: q rotated in place, k and v into the pages) and one
+lbm_attend_frame (paged attention on persistent CTAs, plus the combine of the units several
+CTAs share), host page-table bookkeeping included.  (Folding the rotation of q into the
+attention instead, lbm_append_frame with q = NULL, moves a third fewer bytes in the append
+but costs the attention more than that saves at these sizes, so it is not what is timed.)  The default workload is the 4096-patch stream (configuration 4):
 8 heads x head_dim 128, bf16, 6 special + 64x64 patch tokens per frame, 96 keyframes,
 scale_frames 4, sliding_window 32.  Inputs are seeded synthetic frames held in HBM before
 timing; a pool of up to 64 distinct frames (1.6 GB here) is larger than L2, so no input is
@@ -102,7 +104,7 @@ def frame_work(cfg, n_frames: int | None = None):
 
     Frame n with m keyframes committed before it sees min(m, S+W)+1 patch pages and 6(m+1)
     special tokens; attention = 4 T N_k H D flops (QK^T and PV); append moves 6 T H D e bytes
-    (read q, k, v; write q, k, v).
+    (read q, k, v; write q rotated in place, k and v into the pages).
     """
     T, H, D, e = cfg.tokens, cfg.heads, cfg.head_dim, cfg.elem_bytes
     flops, nbytes, keys = [], [], []

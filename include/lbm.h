@@ -178,7 +178,13 @@ LBM_API int lbm_cache_create_blocks(int num_blocks, int heads, int head_dim,
 /* Rotate and append one frame.  [3DRoPE-KV] "Frame Appending and Position Encoding
  * Integration" and "Complex-Valued Tensor Application"; [VideoRoPE] "Temporal Consistency
  * in KV-Cache Streaming" (t = absolute frame index).
- *   q      device, [T][heads][head_dim]; rotated IN PLACE (read, rotated, written back)
+ *   q      device, [T][heads][head_dim], or NULL.  Non-NULL: rotated IN PLACE by this call
+ *          (read, rotated, written back), and the attention then uses it as it is.  NULL
+ *          (bf16 caches only, else LBM_ERR_UNSUPPORTED): the rotation of q is folded into
+ *          the attention, which rotates the raw q as it loads it ([3DRoPE-KV] FAQ "Where does
+ *          the RoPE application occur relative to the KV cache write?": q is rotated before
+ *          the attention, k before the cache write) and leaves q unchanged; this call then
+ *          moves only k and v (4 instead of 6 x T x heads x head_dim elements).
  *   k, v   device, [T][heads][head_dim]; k is rotated, v is not; both are written into the
  *          frame's patch page (tokens >= 6) and the next 6 slots of the special stream
  *   frame_idx    strictly greater than the previous frame's, and < rope's ppf
@@ -202,18 +208,27 @@ LBM_API int lbm_append_frame_block(lbm_cache_t* cache, int block_idx, void* q, c
                                    const void* v, long long frame_idx, int is_keyframe,
                                    void* stream);
 
-/* Attention of the pending frame's (already rotated) queries over what the cache retains:
- * scale pages -> window pages (oldest first) -> the frame's own page -> all special tokens
- * ([3DRoPE-KV] "Attention Computation with Cached RoPE"); a frame's own tokens all see each
- * other; softmax scale 1/sqrt(head_dim).  Then commits the frame (keyframe; deferred
- * eviction) or rolls it back ([KVBenefits] "Dynamic Keyframe Selection"); a frame appended
- * with LBM_KEYFRAME_DEFERRED stays pending until lbm_commit_frame.
- *   q    device [T][heads][head_dim], the q rotated by lbm_append_frame
+/* Attention of the pending frame's queries over what the cache retains: scale pages ->
+ * window pages (oldest first) -> the frame's own page -> all special tokens ([3DRoPE-KV]
+ * "Attention Computation with Cached RoPE"); a frame's own tokens all see each other; softmax
+ * scale 1/sqrt(head_dim).  Then commits the frame (keyframe; deferred eviction) or rolls it
+ * back ([KVBenefits] "Dynamic Keyframe Selection"); a frame appended with
+ * LBM_KEYFRAME_DEFERRED stays pending until lbm_commit_frame.
+ *   q    device [T][heads][head_dim]: the q lbm_append_frame rotated, or, when the append
+ *        was given q = NULL, the raw q, which the kernel rotates as it loads it (q is not
+ *        written)
  *   out  device [T][heads][head_dim], written
  * bf16: one tcgen05 kernel launch, plus one combine launch when the keys are split across
  * CTAs.  Errors: LBM_ERR_SEQUENCE if no frame is pending or the pending frame has already
  * been attended. */
 LBM_API int lbm_attend_frame(lbm_cache_t* cache, const void* q, void* out, void* stream);
+/* As lbm_attend_frame for a frame whose append left q to the attention (q = NULL there),
+ * and the kernel also writes the rotated q it used, rounded to bf16, into q_rot_out (device
+ * [T][heads][head_dim], caller-owned): what lbm_append_frame would have written into q in
+ * place.  For checks of the folded rotation.  LBM_ERR_INVALID if q_rot_out is NULL or
+ * misaligned, or the frame's q was rotated by its append, or the cache is not bf16. */
+LBM_API int lbm_attend_frame_qrot(lbm_cache_t* cache, const void* q, void* out, void* q_rot_out,
+                                  void* stream);
 /* The same for block block_idx (LBM_ERR_SEQUENCE unless it has just appended). */
 LBM_API int lbm_attend_frame_block(lbm_cache_t* cache, int block_idx, const void* q, void* out,
                                    void* stream);
@@ -299,6 +314,19 @@ LBM_API int lbm_cache_read_kv_block(const lbm_cache_t* cache, int block_idx, int
 /* Synchronises the device and reports a bounded wait that ran out in an earlier kernel
  * (LBM_ERR_TIMEOUT, after which the error word is cleared) or LBM_OK. */
 LBM_API int lbm_cache_check(lbm_cache_t* cache);
+
+/* Time limit of each wait inside the attention kernel's roles (the producer waiting for a
+ * free ring stage, the MMA issuers for loaded tiles and softmax results, the softmax threads
+ * for scores), in nanoseconds of %globaltimer: a wait that runs out sets the device error
+ * word and makes every role of the CTA leave; lbm_cache_check then reports LBM_ERR_TIMEOUT
+ * and the frame's output is not valid.  The waits at the kernel's exit, for copies and
+ * tensor-core operations already issued, keep their own 2 s bound, so nothing is left in
+ * flight when the tensor memory is freed.  Below 1000 ns a wait that is not satisfied at its
+ * first test runs out at once (a waiting thread may sleep longer than that inside one test,
+ * so shorter limits are not honoured literally): the way to exercise the failure path.
+ * ns = 0 restores the default, 2 s (2e9); values above it are LBM_ERR_INVALID.  Host-only;
+ * applies to attention calls made after it. */
+LBM_API int lbm_cache_set_wait_limit(lbm_cache_t* cache, unsigned long long ns);
 
 LBM_API void lbm_cache_destroy(lbm_cache_t* cache);
 

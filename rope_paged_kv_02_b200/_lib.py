@@ -35,8 +35,10 @@ SYMBOLS = [
     "lbm_rope3d_tables", "lbm_rope3d_tables_fhw", "lbm_rope2d_tables", "lbm_rope3d_expand",
     "lbm_rope_destroy",
     "lbm_cache_create", "lbm_cache_create_blocks", "lbm_append_frame", "lbm_append_frame_block",
-    "lbm_attend_frame", "lbm_attend_frame_block", "lbm_attend_frame_noalloc",
+    "lbm_attend_frame", "lbm_attend_frame_block", "lbm_attend_frame_qrot",
+    "lbm_attend_frame_noalloc",
     "lbm_commit_frame", "lbm_cache_reset", "lbm_cache_read_kv_block",
+    "lbm_cache_set_wait_limit",
     "lbm_cache_state", "lbm_cache_read_kv", "lbm_cache_check", "lbm_cache_destroy",
     "lbm_status_string",
     "lbm_pager_create", "lbm_pager_append", "lbm_pager_visible", "lbm_pager_finish",
@@ -106,11 +108,13 @@ def load() -> ctypes.CDLL:
     lib.lbm_append_frame.argtypes = [c_void, c_void, c_void, c_void, c_ll, c_int, c_void]
     lib.lbm_attend_frame.argtypes = [c_void, c_void, c_void, c_void]
     lib.lbm_attend_frame_noalloc.argtypes = [c_void, c_void, c_void, c_void]
+    lib.lbm_attend_frame_qrot.argtypes = [c_void, c_void, c_void, c_void, c_void]
     lib.lbm_commit_frame.argtypes = [c_void, c_int]
     lib.lbm_cache_reset.argtypes = [c_void]
     lib.lbm_cache_state.argtypes = [c_void, ctypes.POINTER(CacheState)]
     lib.lbm_cache_read_kv.argtypes = [c_void, c_int, c_int, c_int, c_void]
     lib.lbm_cache_check.argtypes = [c_void]
+    lib.lbm_cache_set_wait_limit.argtypes = [c_void, ctypes.c_ulonglong]
     lib.lbm_cache_destroy.argtypes = [c_void]
     lib.lbm_cache_destroy.restype = None
     lib.lbm_status_string.argtypes = [c_int]
@@ -265,7 +269,8 @@ class PagedKVCache:
         return self.psi + self.patches
 
     def append_frame(self, q, k, v, frame_idx: int, is_keyframe, stream=None) -> None:
-        """is_keyframe: True / False, or None to decide after attention (commit_frame)."""
+        """is_keyframe: True / False, or None to decide after attention (commit_frame).
+        q: rotated in place here, or None to leave its rotation to attend_frame."""
         _check(load().lbm_append_frame(self.handle, _ptr(q), _ptr(k), _ptr(v), int(frame_idx),
                                        _keyframe_mode(is_keyframe), _stream(stream)),
                "lbm_append_frame")
@@ -283,9 +288,15 @@ class PagedKVCache:
     def commit_frame(self, keep: bool) -> None:
         _check(load().lbm_commit_frame(self.handle, 1 if keep else 0), "lbm_commit_frame")
 
-    def attend_frame(self, q, out, stream=None) -> None:
-        _check(load().lbm_attend_frame(self.handle, _ptr(q), _ptr(out), _stream(stream)),
-               "lbm_attend_frame")
+    def attend_frame(self, q, out, stream=None, q_rot_out=None) -> None:
+        """q_rot_out: also receive the rotated q the kernel used (frames appended with
+        q = None only; lbm_attend_frame_qrot)."""
+        if q_rot_out is None:
+            _check(load().lbm_attend_frame(self.handle, _ptr(q), _ptr(out), _stream(stream)),
+                   "lbm_attend_frame")
+        else:
+            _check(load().lbm_attend_frame_qrot(self.handle, _ptr(q), _ptr(out), _ptr(q_rot_out),
+                                                _stream(stream)), "lbm_attend_frame_qrot")
 
     def reset(self) -> None:
         _check(load().lbm_cache_reset(self.handle), "lbm_cache_reset")
@@ -306,6 +317,11 @@ class PagedKVCache:
 
     def check(self) -> None:
         _check(load().lbm_cache_check(self.handle), "lbm_cache_check")
+
+    def set_wait_limit(self, ns: int) -> None:
+        """lbm_cache_set_wait_limit: bound of each wait of the attention kernel's roles
+        (0: the default, 2 s)."""
+        _check(load().lbm_cache_set_wait_limit(self.handle, int(ns)), "lbm_cache_set_wait_limit")
 
     def close(self) -> None:
         if self.handle:

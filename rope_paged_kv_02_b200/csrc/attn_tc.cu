@@ -7,8 +7,9 @@
 //
 // One CTA = two query tiles of 128 rows of one head, over one split of the key tiles.
 // Both query tiles share every K/V tile the CTA loads.  Warp roles (12 warps):
-//   warp 0      TMA producer: the two Q tiles once, then K/V tiles gathered page by page
-//               through the page table into a ring of shared-memory stages (128B swizzle).
+//   warp 0      TMA producer: the two Q tiles once per segment, then K/V tiles gathered
+//               page by page through the page table into a ring of shared-memory stages
+//               (128B swizzle).
 //   warp 1, 2   allocate tensor memory (warp 1); one lane of warp 1+g issues every
 //               tcgen05.mma of query tile g:
 //                 S = Q_g K_j^T   (A, B from shared memory)      -> TMEM S_g
@@ -20,6 +21,11 @@
 //               row (its TMEM lane); reads S_j, row max, exp2, row sum in fp32, writes P_j
 //               (bf16) into TMEM, and rescales O only when the running max grew by more than
 //               2^8 (lazy rescale; exact because O and l share one reference max).
+//               When the frame's q is raw (its append left q alone), each softmax thread
+//               also rotates its own query row in place in shared memory at the token's
+//               (t, h, w) position before Q.K^T reads it ([3DRoPE-KV] FAQ "Where does the
+//               RoPE application occur relative to the KV cache write?"): the next segment's
+//               rows are rotated while the current segment's last P.V runs.
 //   The two softmax warpgroups run concurrently, so one's exponentials overlap the other's
 //   tensor-core work.
 // Tensor memory: 256 columns per query tile g at 256 g.  head_dim 64, 128-key tiles: S [0,128),
@@ -40,12 +46,13 @@ constexpr int BM = 128;         // query rows per CTA
 constexpr int kThreads = 384;   // 12 warps
 constexpr uint32_t kTmemCols = 512;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+constexpr unsigned long long kImmediateLimitNs = 1000ull;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when max grows by > 2^8
 constexpr unsigned kFull = 0xffffffffu;
 
 constexpr int kMaxStages = 4;  // K/V ring stages the barrier block has room for
 
-template <int D>
+template <int D, bool FOLD>
 struct Cfg {
   static constexpr int BN = attn_key_tile(D);            // keys per K/V tile
   static constexpr int NS = 4;                           // K/V pipeline stages
@@ -60,7 +67,10 @@ struct Cfg {
   static constexpr int OFF_V = OFF_K + NS * KV_TILE;
   static constexpr int OFF_BAR = OFF_V + NS * KV_TILE;
   static constexpr int BAR_BYTES = 256;
-  static constexpr int SMEM = OFF_BAR + BAR_BYTES + 1024;  // + slack to align the base to 1 KB
+  static constexpr int OFF_TAB = OFF_BAR + BAR_BYTES;    // RoPE tables for the q rotation
+  static constexpr int TAB_BYTES = FOLD ? kRopeStageBytes : 0;
+  static constexpr int SMEM = OFF_TAB + TAB_BYTES + 1024;  // + slack to align the base to 1 KB
+  static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
 };
 
 // ---- PTX wrappers -----------------------------------------------------------------------
@@ -104,30 +114,59 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-suspending check of a phase (no wait at all).
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 __device__ __forceinline__ unsigned long long global_timer() {
   unsigned long long t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
 
+// What a bounded wait needs: the CTA's abort flag, the device error word and the time limit
+// of one wait (roles' waits: the cache's wait limit, 2 s unless set; the drains at the exit
+// always use kWaitLimitNs).
+struct WaitCtx {
+  volatile int* abort_flag;
+  int* err;
+  unsigned long long limit_ns;
+};
+
 // Bounded wait for the phase of `bar` with the given parity to complete.  Returns false
 // when the CTA is aborting or the limit ran out (then the error word and abort flag are set).
-__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                       int* err, int where) {
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, WaitCtx wa,
+                                            int where) {
+  if (wa.limit_ns < kImmediateLimitNs) {
+    // a limit below the resolution a suspended try_wait can honour: a wait that is not
+    // satisfied at its first test runs out at once (how the failure path is exercised)
+    *wa.abort_flag = 1;
+    atomicExch(wa.err, where);
+    return false;
+  }
   const unsigned long long t0 = global_timer();
   while (true) {
     if (mbar_try(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (global_timer() - t0 > kWaitLimitNs) {
-      *abort_flag = 1;
-      atomicExch(err, where);
+    if (*wa.abort_flag) return false;
+    if (global_timer() - t0 > wa.limit_ns) {
+      *wa.abort_flag = 1;
+      atomicExch(wa.err, where);
       return false;
     }
   }
 }
 
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          int* err, int where) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtx& wa,
+                                          int where) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
@@ -137,14 +176,14 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
       : "r"(bar), "r"(parity)
       : "memory");
   if (ok) return true;
-  return mbar_wait_slow(bar, parity, abort_flag, err, where);
+  return mbar_wait_slow(bar, parity, wa, where);
 }
 
 // Whole-warp wait: every lane waits, and the vote makes the outcome warp-uniform, so the
 // warp-collective issue helpers after it always run with the full warp.
-__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity,
-                                               volatile int* abort_flag, int* err, int where) {
-  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, err, where));
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, const WaitCtx& wa,
+                                               int where) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, wa, where));
 }
 
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* tm, int x, int y,
@@ -312,7 +351,8 @@ __device__ __forceinline__ TileRef tile_ref(const AttnParams& p, int t) {
 }
 
 struct Bars {
-  uint64_t q_full;         // the query tiles of the current segment landed
+  uint64_t q_loaded;       // the query tiles of the current segment landed (TMA)
+  uint64_t q_full[2];      // per tile g: its rows rotated in place and visible to the MMA (128)
   uint64_t q_empty;        // both MMA issuers are done with them (count 2)
   uint64_t s_full[2][2];   // per query tile g and S buffer: S_j landed in TMEM
   uint64_t s_free[2];      // per g: the softmax warps have read S_j
@@ -367,18 +407,87 @@ __device__ __forceinline__ int seg_nq(const AttnParams& p, const Segment& sg, in
   return min(2, q_tiles - 2 * seg_pair(p, sg));
 }
 
+// One query row in shared memory (K-major, 128-byte swizzle as the TMA box leaves it: the
+// 16-byte chunk c of row r of an atom sits at chunk position c ^ (r % 8); the next 64
+// features are one atom further) put in final form by its own thread.  With p.rotate_q the
+// row's feature pairs are rotated at the token's (t, h, w) position in fp32 and rounded once
+// to bf16 ([3DRoPE-KV] "Complex-Valued Tensor Application"), the same arithmetic as the
+// append kernel's, and written back in place; with p.q_rot_out (first segment of the unit
+// only: one writer per row) the rotated row is also stored there.  The (cos, sin) pairs come
+// from the CTA's shared-memory copy of the tables (tab: t row of the frame, then the h and w
+// tables) when p.rope_staged, else from global memory.  Rows past the frame are zeros from
+// the TMA and stay zeros.  Ends with the fence that makes the generic-proxy writes visible to
+// the tensor core.  Not inlined: it runs once per segment, and its registers stay out of the
+// softmax loop's budget.
+template <int D, int Q_ATOM>
+__device__ __noinline__ void place_q_row(const AttnParams& p, const float2* tab, uint32_t q_row,
+                                         int row, int head, bool writer) {
+  if (!p.rotate_q || row >= p.tokens) return;
+  const RopeTables& rt = p.rope;
+  int hh = 0, ww = 0;
+  if (row >= rt.psi) {
+    const int pj = row - rt.psi;
+    hh = 1 + pj / rt.ppw;
+    ww = 1 + pj - (hh - 1) * rt.ppw;
+  }
+  // the row of each axis table this token uses
+  const bool staged = p.rope_staged != 0;
+  const float2* bt = staged ? tab : rt.tab_t + (size_t)p.frame * rt.nt;
+  const float2* bh = staged ? tab + rt.nt + hh * rt.nh : rt.tab_h + (size_t)hh * rt.nh;
+  const float2* bw = staged ? tab + rt.nt + (rt.pph + 1) * rt.nh + ww * rt.nw
+                            : rt.tab_w + (size_t)ww * rt.nw;
+  const int nth = rt.nt + rt.nh;
+  const uint32_t sw = (uint32_t)(row & 7);  // the swizzle phase of this row (row % 8 of the tile)
+  uint4* out = p.q_rot_out != nullptr && writer
+                   ? reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.q_rot_out) +
+                                              ((size_t)row * p.heads + head) * D)
+                   : nullptr;
+#pragma unroll
+  for (int a = 0; a < D / 64; ++a) {
+    float2 cs[32];
+#pragma unroll
+    for (int u = 0; u < 32; ++u) {
+      const int i = 32 * a + u;
+      cs[u] = i < rt.nt ? bt[i] : (i < nth ? bh[i - rt.nt] : bw[i - nth]);
+    }
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const uint32_t addr = q_row + a * Q_ATOM + ((c ^ sw) << 4);
+      uint32_t w[4];
+      asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                   : "r"(addr));
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float2 r = cs[4 * c + u];
+        const float x0 = __uint_as_float(w[u] << 16), x1 = __uint_as_float(w[u] & 0xffff0000u);
+        w[u] = pack_bf16(fmaf(x0, r.x, -x1 * r.y), fmaf(x0, r.y, x1 * r.x));
+      }
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[0]),
+                   "r"(w[1]), "r"(w[2]), "r"(w[3])
+                   : "memory");
+      if (out != nullptr) out[8 * a + c] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+  // generic-proxy writes, read by the tensor core through the async proxy
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Persistent CTA c of p.grid walks the global work items [sk_start[c], sk_start[c+1]).  Every role
 // walks the same segments; barrier phases run on across segments (counters per role).
-template <int D>
+// FOLD: the frame's q is raw and every softmax thread rotates its query row in place after the
+// TMA load (the append left q alone); without it the q rows are used as loaded.
+template <int D, bool FOLD>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ AttnParams p) {
-  using C = Cfg<D>;
+  using C = Cfg<D, FOLD>;
   using TM = TmemMap<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   Bars* bars = reinterpret_cast<Bars*>(smem + C::OFF_BAR);
   volatile int* abort_flag = &bars->abort_flag;
+  const WaitCtx wa{abort_flag, p.err, p.wait_limit_ns};
 
   // warp index through a shuffle: provably warp-uniform, so role-dependent descriptors and
   // addresses stay in uniform registers
@@ -394,7 +503,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar = [&](const uint64_t& b) { return smem_u32(&b); };
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(bars->q_full), 1);
+    mbar_init(bar(bars->q_loaded), 1);
+    mbar_init(bar(bars->q_full[0]), 128);
+    mbar_init(bar(bars->q_full[1]), 128);
     mbar_init(bar(bars->q_empty), 2);
     for (int g = 0; g < 2; ++g) {
       for (int b = 0; b < 2; ++b) {
@@ -412,6 +523,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     bars->abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  // the frame's row of the t table and the whole h and w tables, for the in-kernel rotation
+  // of q (constant inputs, so this may overlap the previous kernel's tail)
+  float2* tab = reinterpret_cast<float2*>(smem + C::OFF_TAB);
+  if (FOLD && p.rope_staged) {
+    const RopeTables& rt = p.rope;
+    const int n_h = (rt.pph + 1) * rt.nh, n_w = (rt.ppw + 1) * rt.nw;
+    for (int i = threadIdx.x; i < rt.nt + n_h + n_w; i += kThreads)
+      tab[i] = i < rt.nt ? __ldg(rt.tab_t + (size_t)p.frame * rt.nt + i)
+                         : (i < rt.nt + n_h ? __ldg(rt.tab_h + (i - rt.nt))
+                                            : __ldg(rt.tab_w + (i - rt.nt - n_h)));
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -438,24 +560,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       x = sg.unit * p.n_tiles + sg.b;
       // the query buffers are free once both MMA issuers are done with the last segment
       if (seg_i > 0 &&
-          !mbar_wait_warp(bar(bars->q_empty), (seg_i - 1) & 1, abort_flag, p.err, 12)) {
+          !mbar_wait_warp(bar(bars->q_empty), (seg_i - 1) & 1, wa, 12)) {
         ok = false;
         break;
       }
       const int n_q = seg_nq(p, sg, q_tiles);
       const int head = seg_head(p, sg);
-      mbar_expect_tx(bar(bars->q_full), n_q * C::Q_TILE);
+      mbar_expect_tx(bar(bars->q_loaded), n_q * C::Q_TILE);
       for (int g = 0; g < n_q; ++g) {
 #pragma unroll
         for (int a = 0; a < C::ATOMS; ++a)
           tma_load_3d(sQ + g * C::Q_TILE + a * C::Q_ATOM, &p.tm_q, 64 * a, head,
-                      (2 * seg_pair(p, sg) + g) * BM, bar(bars->q_full));
+                      (2 * seg_pair(p, sg) + g) * BM, bar(bars->q_loaded));
       }
       for (int t = sg.a; t < sg.b; ++t, ++issued) {
         const int s = issued % C::NS;
         if (issued >= C::NS &&
-            !mbar_wait_warp(bar(bars->kv_empty[s]), ((issued - C::NS) / C::NS) & 1, abort_flag,
-                            p.err, 1)) {
+            !mbar_wait_warp(bar(bars->kv_empty[s]), ((issued - C::NS) / C::NS) & 1, wa,
+                             1)) {
           ok = false;
           break;
         }
@@ -476,7 +598,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // drain: wait (bounded) for the copies this warp issued that may still be landing
       if (seg_i > 0) {
         const unsigned long long t0 = global_timer();
-        while (!mbar_try(bar(bars->q_full), (seg_i - 1) & 1) &&
+        while (!mbar_try(bar(bars->q_loaded), (seg_i - 1) & 1) &&
                global_timer() - t0 < kWaitLimitNs) {
         }
       }
@@ -504,7 +626,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Segment sg = segment_at(p, x, hi);
       x = sg.unit * p.n_tiles + sg.b;
       const int n = sg.b - sg.a;
-      if (!mbar_wait_warp(bar(bars->q_full), seg_i & 1, abort_flag, p.err, 2)) {
+      if (!mbar_wait_warp(bar(bars->q_loaded), seg_i & 1, wa, 2)) {
         ok = false;
         break;
       }
@@ -513,7 +635,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // after the tile has landed, so no arrival can run a phase ahead
         for (int t = 0; t < n; ++t, ++ring) {
           const int s = ring % C::NS;
-          if (!mbar_wait_warp(bar(bars->kv_full[s]), (ring / C::NS) & 1, abort_flag, p.err, 4)) {
+          if (!mbar_wait_warp(bar(bars->kv_full[s]), (ring / C::NS) & 1, wa, 4)) {
             ok = false;
             break;
           }
@@ -522,21 +644,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(bar(bars->q_empty));
         continue;
       }
+      // this tile's rows are in final form: rotated in place by the softmax threads when q is
+      // raw (when it was rotated by the append, the TMA load alone is enough)
+      if (FOLD && !mbar_wait_warp(bar(bars->q_full[g]), segs & 1, wa, 14)) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
       const int j0 = jg;  // first tile of this segment in this query tile's count
       auto issue_qk = [&](int j) -> bool {
         const int s = (ring + (j - j0)) % C::NS;
         const int r = ring + (j - j0);
-        if (!mbar_wait_warp(bar(bars->kv_full[s]), (r / C::NS) & 1, abort_flag, p.err, 4))
+        if (!mbar_wait_warp(bar(bars->kv_full[s]), (r / C::NS) & 1, wa, 4))
           return false;
         // the S buffer of tile j is free: one buffer, the softmax has read S_{j-1}; two
         // buffers, PV_{j-2} has read P_{j-2}, which was written after S_{j-2} was read
         if (TM::NB == 1) {
           if (j >= 1 &&
-              !mbar_wait_warp(bar(bars->s_free[g]), (j - 1) & 1, abort_flag, p.err, 5))
+              !mbar_wait_warp(bar(bars->s_free[g]), (j - 1) & 1, wa, 5))
             return false;
         } else if (j >= 2 && !mbar_wait_warp(bar(bars->pv_done[g][TM::buf(j)]), TM::par(j - 2),
-                                             abort_flag, p.err, 5)) {
+                                             wa, 5)) {
           return false;
         }
         tc_fence_after();
@@ -553,11 +681,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
       auto issue_pv = [&](int i) -> bool {
-        if (!mbar_wait_warp(bar(bars->p_full[g][TM::buf(i)]), TM::par(i), abort_flag, p.err, 3))
+        if (!mbar_wait_warp(bar(bars->p_full[g][TM::buf(i)]), TM::par(i), wa, 3))
           return false;
         // O of the previous segment must have been read out before the first PV overwrites it
         if (i == j0 && segs > 0 &&
-            !mbar_wait_warp(bar(bars->o_free[g]), (segs - 1) & 1, abort_flag, p.err, 13))
+            !mbar_wait_warp(bar(bars->o_free[g]), (segs - 1) & 1, wa, 13))
           return false;
         tc_fence_after();
         const int s = (ring + (i - j0)) % C::NS;
@@ -603,10 +731,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     int jg = 0;
     int seg_i = 0;
     bool ok = true;
+    bool q_placed = false;  // this segment's rows were placed ahead, during the last one
+    // waits for segment k's query tiles and, if this tile takes part, puts its row in final
+    // form; every segment's q_loaded phase is waited, so its parity stays unambiguous
+    auto place_q = [&](const Segment& qs, int k) -> bool {
+      if (!FOLD) return true;  // q rotated by the append: nothing to place
+      if (!__all_sync(kFull, mbar_wait(bar(bars->q_loaded), k & 1, wa, 15)))
+        return false;
+      if (g < seg_nq(p, qs, q_tiles)) {
+        // this thread's row of tile g (recomputed here: nothing of it stays live in the loop)
+        const uint32_t q_row = smem_u32(smem + C::OFF_Q) + g * C::Q_TILE +
+                               ((threadIdx.x - 128u) & 127u) * 128u;
+        place_q_row<D, C::Q_ATOM>(p, reinterpret_cast<const float2*>(smem + C::OFF_TAB), q_row,
+                                   (2 * seg_pair(p, qs)) * BM + row_in_pair, seg_head(p, qs),
+                                   qs.a == 0);
+        mbar_arrive(bar(bars->q_full[g]));
+      }
+      return true;
+    };
     uint32_t S[BN];
     for (int x = lo; ok && x < hi; ++seg_i) {
       const Segment sg = segment_at(p, x, hi);
       x = sg.unit * p.n_tiles + sg.b;
+      if (FOLD && !q_placed && !place_q(sg, seg_i)) {
+        ok = false;
+        break;
+      }
+      q_placed = false;
       if (g >= seg_nq(p, sg, q_tiles)) continue;
       const int n = sg.b - sg.a;
       const int j0 = jg;
@@ -618,7 +769,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int sb = TM::buf(j);
         const uint32_t tS = lane_base + TM::S(sb);
         const uint32_t tP = lane_base + TM::P(sb);
-        if (!__all_sync(kFull, mbar_wait(bar(bars->s_full[g][sb]), TM::par(j), abort_flag, p.err,
+        if (!__all_sync(kFull, mbar_wait(bar(bars->s_full[g][sb]), TM::par(j), wa, 
                                          6))) {
           ok = false;
           break;
@@ -660,8 +811,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // one P buffer: P_j overwrites P_{j-1}, so PV_{j-1} must have finished (two buffers:
         // P_j goes to its own S buffer; PV_{j-1} is waited for only before rescaling O)
         if (TM::NB == 1 && j >= 1 &&
-            !__all_sync(kFull, mbar_wait(bar(bars->pv_done[g][0]), (j - 1) & 1, abort_flag,
-                                         p.err, 7))) {
+            !__all_sync(kFull, mbar_wait(bar(bars->pv_done[g][0]), (j - 1) & 1, wa,
+                                          7))) {
           ok = false;
           break;
         }
@@ -698,7 +849,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // O holds sum_{i<j} P_i V_i relative to the old max: scale it before PV_j lands
           if (TM::NB == 2 &&
               !__all_sync(kFull, mbar_wait(bar(bars->pv_done[g][TM::buf(j - 1)]),
-                                           TM::par(j - 1), abort_flag, p.err, 7))) {
+                                           TM::par(j - 1), wa, 7))) {
             ok = false;
             break;
           }
@@ -719,10 +870,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         mbar_arrive(bar(bars->p_full[g][sb]));
       }
+      // the next segment's query tiles land once both Q.K^T of this one are done: if they
+      // are there, put them in final form now, while the last P.V of this segment runs
+      // (otherwise at the top of the next segment, after this one's epilogue)
+      if (FOLD && ok && x < hi &&
+          __all_sync(kFull, mbar_test(bar(bars->q_loaded), (seg_i + 1) & 1))) {
+        if (!place_q(segment_at(p, x, hi), seg_i + 1)) {
+          ok = false;
+          break;
+        }
+        q_placed = true;
+      }
       jg += n;
       if (!ok ||
           !__all_sync(kFull, mbar_wait(bar(bars->pv_done[g][TM::buf(jg - 1)]), TM::par(jg - 1),
-                                       abort_flag, p.err,
+                                       wa, 
                                        9))) {
         ok = false;
         break;
@@ -902,18 +1064,19 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const __grid_constant
 
 }  // namespace
 
-size_t attn_tc_smem_bytes(int head_dim) {
-  return head_dim == 64 ? Cfg<64>::SMEM : Cfg<128>::SMEM;
+size_t attn_tc_smem_bytes(int head_dim, bool fold) {
+  if (head_dim == 64) return fold ? Cfg<64, true>::SMEM : Cfg<64, false>::SMEM;
+  return fold ? Cfg<128, true>::SMEM : Cfg<128, false>::SMEM;
 }
 
 namespace {
 
-template <int D>
+template <int D, bool FOLD>
 cudaError_t prepare_attn_tc() {
   static cudaError_t state = cudaErrorNotReady;
   if (state == cudaErrorNotReady)
-    state = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 Cfg<D>::SMEM);
+    state = cudaFuncSetAttribute(attn_tc_kernel<D, FOLD>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D, FOLD>::SMEM);
   return state;
 }
 
@@ -940,19 +1103,21 @@ cudaError_t launch_pdl(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_
   return cudaLaunchKernelEx(&cfg, kernel, p);
 }
 
+template <int D, bool FOLD>
+cudaError_t launch_attn_tc_t(const AttnParams& p, cudaStream_t s) {
+  cudaError_t e;
+  if ((e = prepare_attn_tc<D, FOLD>()) != cudaSuccess) return e;
+  return launch_pdl(attn_tc_kernel<D, FOLD>, dim3(p.grid), dim3(kThreads), Cfg<D, FOLD>::SMEM,
+                    s, p);
+}
+
 }  // namespace
 
 cudaError_t launch_attn_tc(const AttnParams& p, int head_dim, cudaStream_t s) {
-  const dim3 grid(p.grid);
-  cudaError_t e;
-  if (head_dim == 64) {
-    if ((e = prepare_attn_tc<64>()) != cudaSuccess) return e;
-    return launch_pdl(attn_tc_kernel<64>, grid, dim3(kThreads), Cfg<64>::SMEM, s, p);
-  }
-  if (head_dim == 128) {
-    if ((e = prepare_attn_tc<128>()) != cudaSuccess) return e;
-    return launch_pdl(attn_tc_kernel<128>, grid, dim3(kThreads), Cfg<128>::SMEM, s, p);
-  }
+  const bool fold = p.rotate_q != 0;
+  if (head_dim == 64) return fold ? launch_attn_tc_t<64, true>(p, s) : launch_attn_tc_t<64, false>(p, s);
+  if (head_dim == 128)
+    return fold ? launch_attn_tc_t<128, true>(p, s) : launch_attn_tc_t<128, false>(p, s);
   return cudaErrorInvalidValue;
 }
 

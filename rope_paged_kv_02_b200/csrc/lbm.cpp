@@ -29,6 +29,8 @@ struct CacheBlock {
   CUtensorMap tm_kp, tm_vp, tm_ks, tm_vs;
 };
 
+constexpr unsigned long long kDefaultWaitLimitNs = 2000000000ull;
+
 struct lbm_cache {
   int heads, head_dim, patches, psi, scale_frames, sliding_window, max_frames, dtype;
   int device = 0;
@@ -43,9 +45,11 @@ struct lbm_cache {
   float* part_lse = nullptr;
   size_t scratch_floats = 0;    // capacity of part_o + part_lse in floats
   int forced_grid = 0;          // LBM_ATTN_GRID at create time (0: one CTA per SM)
+  unsigned long long wait_limit_ns = kDefaultWaitLimitNs;  // lbm_cache_set_wait_limit
   int* d_err = nullptr;
   long long device_bytes = 0;
   long long launches = 0;       // kernels launched so far
+  bool q_rotated = false;       // the pending block's q was rotated by its append
   CUtensorMap tm_q;             // cached for the last q pointer seen
   const void* tm_q_ptr = nullptr;
   lbm::Pager pager;
@@ -113,7 +117,8 @@ void order_after(lbm_cache* c, cudaStream_t s) {
 // Fills everything of the attention parameters but the partial-result scratch: the visible
 // page list (no container), tensor maps, and the stream-K partition of the frame's work
 // over the persistent CTAs.  Returns LBM_OK or an error status.
-int fill_attn_params(lbm_cache* c, int block, const void* q, void* out, lbm::AttnParams& p) {
+int fill_attn_params(lbm_cache* c, int block, const void* q, void* out, void* q_rot_out,
+                     lbm::AttnParams& p) {
   const CacheBlock& bk = c->blocks[block];
   int n_pages = 0;
   for (const auto& e : c->pager.scale()) p.pages[n_pages++] = (uint16_t)e.page;
@@ -128,12 +133,18 @@ int fill_attn_params(lbm_cache* c, int block, const void* q, void* out, lbm::Att
     c->tm_q_ptr = q;
   }
   p.tm_q = c->tm_q;
+  p.q_rot_out = q_rot_out;
+  p.rope = c->rope->t;
+  p.rotate_q = c->q_rotated ? 0 : 1;
+  p.rope_staged = p.rotate_q && lbm::rope_fits_stage(c->rope->t) ? 1 : 0;
+  p.frame = (int)c->pager.pending_frame();
   p.tm_kp = bk.tm_kp;
   p.tm_vp = bk.tm_vp;
   p.tm_ks = bk.tm_ks;
   p.tm_vs = bk.tm_vs;
   p.out = out;
   p.err = c->d_err;
+  p.wait_limit_ns = c->wait_limit_ns;
   p.tokens = T;
   p.heads = c->heads;
   p.patches = c->patches;
@@ -213,6 +224,78 @@ int build_rope(lbm::RopeTables t, AxisSpec at, AxisSpec ah, AxisSpec aw, lbm_rop
   t.tab_w = r->d_tables + n_t + n_h;
   r->t = t;
   *out = r;
+  return LBM_OK;
+}
+
+// Attention of block `block` of the pending frame, then its commit / rollback when it is the
+// last block.  q_rot_out: where the kernel also writes the q it rotated (nullable; only when
+// it rotates).  noalloc: partial results in the library's file-scope array instead of the
+// cache's scratch (lbm_attend_frame_noalloc).
+int attend(lbm_cache* c, int block, const void* q, void* out, void* q_rot_out, bool noalloc,
+           void* stream) {
+  if (!c || !q || !out || !aligned16(q) || !aligned16(out)) return LBM_ERR_INVALID;
+  if (block < 0 || block >= (int)c->blocks.size()) return LBM_ERR_INVALID;
+  if (block != c->next_block || !c->block_appended || !c->pager.awaiting_attention())
+    return LBM_ERR_SEQUENCE;
+  if (q_rot_out && (c->q_rotated || c->dtype != LBM_BF16)) return LBM_ERR_INVALID;
+  const lbm::Pools& pl = c->blocks[block].pools;
+  if (use_device(c->device) != LBM_OK) return LBM_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int T = c->psi + c->patches;
+  if (c->dtype == LBM_BF16) {
+    // nothing on this path touches the heap (the no-allocation call relies on it): the
+    // parameter block (~7 KB) lives on the stack and the page list is read in place
+    float* scratch = c->part_o;
+    size_t scratch_floats = c->scratch_floats;
+    if (noalloc) {
+      const int st = lbm::noalloc_scratch(c->device, &scratch, &scratch_floats);
+      if (st != LBM_OK) return st;
+    }
+    lbm::AttnParams p;
+    const int st = fill_attn_params(c, block, q, out, q_rot_out, p);
+    if (st != LBM_OK) return st;
+    const long long units = (long long)p.n_pairs * c->heads;
+    const bool split = lbm::sk_has_split(p);
+    if (split && lbm::sk_scratch_floats(units, p.grid, c->head_dim) > scratch_floats)
+      return LBM_ERR_CAPACITY;
+    p.part_o = scratch;
+    p.part_lse = noalloc ? scratch + (size_t)(units + p.grid) * 256 * c->head_dim : c->part_lse;
+    order_before(c, s);
+    if (lbm::launch_attn_tc(p, c->head_dim, s) != cudaSuccess) return LBM_ERR_CUDA;
+    ++c->launches;
+    if (split) {
+      if (lbm::launch_attn_combine(p, c->head_dim, s) != cudaSuccess) return LBM_ERR_CUDA;
+      ++c->launches;
+    }
+  } else {
+    std::vector<int> pages;
+    int n_sp = 0, last_len = 0;
+    if (c->pager.visible(&pages, &n_sp, &last_len) != lbm::PagerStatus::kOk)
+      return LBM_ERR_SEQUENCE;
+    static thread_local lbm::SimtParams p;
+    p.q = q;
+    p.out = out;
+    p.k_patch = pl.k_patch;
+    p.v_patch = pl.v_patch;
+    p.k_special = pl.k_special;
+    p.v_special = pl.v_special;
+    p.tokens = T;
+    p.heads = c->heads;
+    p.head_dim = c->head_dim;
+    p.patches = c->patches;
+    p.page_stride = pl.page_stride;
+    p.pool_pages = pl.num_pages;
+    p.spec_cap = pl.spec_cap;
+    p.n_pages = (int)pages.size();
+    p.n_special = n_sp;
+    p.scale = (float)(1.0 / std::sqrt((double)c->head_dim));
+    for (size_t i = 0; i < pages.size(); ++i) p.pages[i] = (uint16_t)pages[i];
+    order_before(c, s);
+    if (lbm::launch_attn_simt(p, s) != cudaSuccess) return LBM_ERR_CUDA;
+    ++c->launches;
+  }
+  order_after(c, s);
+  block_attended(c);
   return LBM_OK;
 }
 
@@ -421,8 +504,10 @@ int lbm_append_frame(lbm_cache_t* c, void* q, const void* k, const void* v, long
 
 int lbm_append_frame_block(lbm_cache_t* c, int block, void* q, const void* k, const void* v,
                            long long frame_idx, int is_keyframe, void* stream) {
-  if (!c || !q || !k || !v || !aligned16(q) || !aligned16(k) || !aligned16(v))
+  if (!c || !k || !v || !aligned16(q) || !aligned16(k) || !aligned16(v))
     return LBM_ERR_INVALID;
+  // q = NULL leaves the rotation of q to the attention kernel (tensor-core path only)
+  if (!q && c->dtype != LBM_BF16) return LBM_ERR_UNSUPPORTED;
   if (is_keyframe < 0 || is_keyframe > LBM_KEYFRAME_DEFERRED) return LBM_ERR_INVALID;
   if (block < 0 || block >= (int)c->blocks.size()) return LBM_ERR_INVALID;
   if (block != c->next_block || c->block_appended) return LBM_ERR_SEQUENCE;
@@ -466,6 +551,7 @@ int lbm_append_frame_block(lbm_cache_t* c, int block, void* q, const void* k, co
     c->frame_mode = is_keyframe;
   }
   c->block_appended = true;
+  c->q_rotated = q != nullptr;
   return LBM_OK;
 }
 
@@ -482,94 +568,24 @@ int lbm_commit_frame(lbm_cache_t* c, int keep) {
 
 int lbm_attend_frame(lbm_cache_t* c, const void* q, void* out, void* stream) {
   if (!c) return LBM_ERR_INVALID;
-  return lbm_attend_frame_block(c, c->next_block, q, out, stream);
+  return attend(c, c->next_block, q, out, nullptr, false, stream);
 }
 
 int lbm_attend_frame_block(lbm_cache_t* c, int block, const void* q, void* out, void* stream) {
-  if (!c || !q || !out || !aligned16(q) || !aligned16(out)) return LBM_ERR_INVALID;
-  if (block < 0 || block >= (int)c->blocks.size()) return LBM_ERR_INVALID;
-  std::vector<int> pages;
-  int n_sp = 0, last_len = 0;
-  if (block != c->next_block || !c->block_appended || !c->pager.awaiting_attention() ||
-      c->pager.visible(&pages, &n_sp, &last_len) != lbm::PagerStatus::kOk)
-    return LBM_ERR_SEQUENCE;
-  const lbm::Pools& pl = c->blocks[block].pools;
-  if (use_device(c->device) != LBM_OK) return LBM_ERR_CUDA;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int T = c->psi + c->patches;
-  order_before(c, s);
-  if (c->dtype == LBM_BF16) {
-    static thread_local lbm::AttnParams p;  // ~7 KB: kept off the stack
-    const int st = fill_attn_params(c, block, q, out, p);
-    if (st != LBM_OK) return st;
-    const long long units = (long long)p.n_pairs * c->heads;
-    if (lbm::sk_scratch_floats(units, p.grid, c->head_dim) > c->scratch_floats)
-      return LBM_ERR_CAPACITY;
-    p.part_o = c->part_o;      // sized for (units + max grid) slots at creation
-    p.part_lse = c->part_lse;
-    if (lbm::launch_attn_tc(p, c->head_dim, s) != cudaSuccess) return LBM_ERR_CUDA;
-    ++c->launches;
-    if (lbm::sk_has_split(p)) {
-      if (lbm::launch_attn_combine(p, c->head_dim, s) != cudaSuccess) return LBM_ERR_CUDA;
-      ++c->launches;
-    }
-  } else {
-    static thread_local lbm::SimtParams p;
-    p.q = q;
-    p.out = out;
-    p.k_patch = pl.k_patch;
-    p.v_patch = pl.v_patch;
-    p.k_special = pl.k_special;
-    p.v_special = pl.v_special;
-    p.tokens = T;
-    p.heads = c->heads;
-    p.head_dim = c->head_dim;
-    p.patches = c->patches;
-    p.page_stride = pl.page_stride;
-    p.pool_pages = pl.num_pages;
-    p.spec_cap = pl.spec_cap;
-    p.n_pages = (int)pages.size();
-    p.n_special = n_sp;
-    p.scale = (float)(1.0 / std::sqrt((double)c->head_dim));
-    for (size_t i = 0; i < pages.size(); ++i) p.pages[i] = (uint16_t)pages[i];
-    if (lbm::launch_attn_simt(p, s) != cudaSuccess) return LBM_ERR_CUDA;
-    ++c->launches;
-  }
-  order_after(c, s);
-  block_attended(c);
-  return LBM_OK;
+  return attend(c, block, q, out, nullptr, false, stream);
+}
+
+int lbm_attend_frame_qrot(lbm_cache_t* c, const void* q, void* out, void* q_rot_out,
+                          void* stream) {
+  if (!c) return LBM_ERR_INVALID;
+  if (!q_rot_out || !aligned16(q_rot_out)) return LBM_ERR_INVALID;
+  return attend(c, c->next_block, q, out, q_rot_out, false, stream);
 }
 
 int lbm_attend_frame_noalloc(lbm_cache_t* c, const void* q, void* out, void* stream) {
-  if (!c || !q || !out || !aligned16(q) || !aligned16(out)) return LBM_ERR_INVALID;
+  if (!c) return LBM_ERR_INVALID;
   if (c->dtype != LBM_BF16) return LBM_ERR_UNSUPPORTED;
-  if (!c->block_appended || !c->pager.awaiting_attention()) return LBM_ERR_SEQUENCE;
-  const int block = c->next_block;
-  if (use_device(c->device) != LBM_OK) return LBM_ERR_CUDA;
-  float* scratch = nullptr;
-  size_t scratch_floats = 0;
-  const int st = lbm::noalloc_scratch(c->device, &scratch, &scratch_floats);
-  if (st != LBM_OK) return st;
-  lbm::AttnParams p;  // on the stack: this call touches no heap
-  const int pst = fill_attn_params(c, block, q, out, p);
-  if (pst != LBM_OK) return pst;
-  const long long units = (long long)p.n_pairs * c->heads;
-  const bool split = lbm::sk_has_split(p);
-  if (split && lbm::sk_scratch_floats(units, p.grid, c->head_dim) > scratch_floats)
-    return LBM_ERR_CAPACITY;
-  p.part_o = scratch;
-  p.part_lse = scratch + (size_t)(units + p.grid) * 256 * c->head_dim;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  order_before(c, s);
-  if (lbm::launch_attn_tc(p, c->head_dim, s) != cudaSuccess) return LBM_ERR_CUDA;
-  ++c->launches;
-  if (split) {
-    if (lbm::launch_attn_combine(p, c->head_dim, s) != cudaSuccess) return LBM_ERR_CUDA;
-    ++c->launches;
-  }
-  order_after(c, s);
-  block_attended(c);
-  return LBM_OK;
+  return attend(c, c->next_block, q, out, nullptr, true, stream);
 }
 
 int lbm_cache_reset(lbm_cache_t* c) {
@@ -621,6 +637,12 @@ int lbm_cache_read_kv_block(const lbm_cache_t* c, int block, int which, int inde
   if (cudaMemcpy2D(host_out, width, src, pitch, width, c->heads, cudaMemcpyDeviceToHost) !=
       cudaSuccess)
     return LBM_ERR_CUDA;
+  return LBM_OK;
+}
+
+int lbm_cache_set_wait_limit(lbm_cache_t* c, unsigned long long ns) {
+  if (!c || ns > kDefaultWaitLimitNs) return LBM_ERR_INVALID;
+  c->wait_limit_ns = ns == 0 ? kDefaultWaitLimitNs : ns;
   return LBM_OK;
 }
 

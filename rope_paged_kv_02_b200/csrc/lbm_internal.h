@@ -39,7 +39,7 @@ struct AppendArgs {
   int frame;          // absolute frame index (t coordinate)
   int page;           // patch page of this frame
   int special_slot;   // first special slot of this frame
-  void* q;            // rotated in place
+  void* q;            // rotated in place; NULL: left to the attention kernel
   const void* k;
   const void* v;
 };
@@ -53,6 +53,15 @@ __host__ __device__ constexpr int attn_key_tile(int head_dim) { return head_dim 
 
 constexpr int kMaxGrid = 1024;  // persistent attention CTAs per launch, at most
 
+// Shared memory the attention kernel sets aside for the RoPE tables of its in-kernel q
+// rotation: the frame's t row and the h and w tables, (nt + (pph+1) nh + (ppw+1) nw) float2.
+// Larger tables are read from global memory instead.
+constexpr int kRopeStageBytes = 24 * 1024;
+inline bool rope_fits_stage(const RopeTables& rt) {
+  return ((long long)rt.nt + (long long)(rt.pph + 1) * rt.nh + (long long)(rt.ppw + 1) * rt.nw) *
+             8 <= kRopeStageBytes;
+}
+
 // Kernel parameter block of the paged attention (passed by value).
 // Stream-K partition of one frame's attention over `grid` persistent CTAs.  A unit is one
 // (pair of 128-row query tiles, head), unit u = head * n_pairs + pair; its key tiles are the
@@ -62,15 +71,21 @@ constexpr int kMaxGrid = 1024;  // persistent attention CTAs per launch, at most
 // partial (O, LSE) into slot unit + c (dense: at most units + grid slots), merged by the
 // combine kernel.  The host places the boundaries by cost (sk_partition).
 struct AttnParams {
-  CUtensorMap tm_q;      // q   {head_dim, heads, T}
+  CUtensorMap tm_q;      // q   {head_dim, heads, T}: raw (rotate_q) or already rotated
   CUtensorMap tm_kp;     // K patch pool {head_dim, P*stride, heads}
   CUtensorMap tm_vp;
   CUtensorMap tm_ks;     // K special pool {head_dim, spec_cap, heads}
   CUtensorMap tm_vs;
+  void* q_rot_out;       // nullable [T][heads][head_dim] bf16: the rotated q the kernel used
+  RopeTables rope;       // tables of the in-kernel rotation of q
+  int rotate_q;          // 1: rotate q at its tokens' positions before Q.K^T
+  int rope_staged;       // 1: the kernel copies the tables to shared memory (they fit)
+  int frame;             // t coordinate of the frame (absolute frame index)
   void* out;             // [T][heads][head_dim] bf16
   float* part_o;         // [units + grid slots][256 rows][head_dim] fp32 partial outputs
   float* part_lse;       // [units + grid slots][256 rows] log2-domain LSE
   int* err;              // device error word (bounded waits)
+  unsigned long long wait_limit_ns;  // limit of one wait of the kernel's roles
   int tokens;            // T
   int heads;
   int patches;           // valid tokens per patch page
@@ -108,7 +123,7 @@ cudaError_t launch_rope_append(const RopeTables& rt, const Pools& pools,
                                const AppendArgs& a, cudaStream_t s);
 
 // attn_tc.cu (bf16, tcgen05)
-size_t attn_tc_smem_bytes(int head_dim);
+size_t attn_tc_smem_bytes(int head_dim, bool fold);
 cudaError_t launch_attn_tc(const AttnParams& p, int head_dim, cudaStream_t s);
 // merges the partial results of every unit that spans more than one CTA
 cudaError_t launch_attn_combine(const AttnParams& p, int head_dim, cudaStream_t s);

@@ -104,7 +104,9 @@ constexpr int kAppendThreads = 256;
 // Lanes run over chunks first, then tokens, so a warp reads whole 128-byte rows of q, k, v
 // and, per head, writes consecutive rows of the frame's page.  All 3 * HG loads of a thread
 // are issued before the first rotation, to keep enough bytes in flight to cover HBM latency.
-template <typename T, int CPR, int HG>
+// WITH_Q = false: q is left to the attention kernel, which rotates it as it loads it; the
+// pass then reads k, v and writes the pools only (4 instead of 6 T H D element moves).
+template <typename T, int CPR, int HG, bool WITH_Q>
 __global__ void __launch_bounds__(kAppendThreads)
     rope_append_kernel(RopeTables rt, Pools pools, AppendArgs a) {
   constexpr int EPC = 16 / sizeof(T);  // elements per 16-byte chunk
@@ -126,7 +128,7 @@ __global__ void __launch_bounds__(kAppendThreads)
   U4 vq[HG], vk[HG], vv[HG];
 #pragma unroll
   for (int u = 0; u < HG; ++u) {
-    vq[u] = ld_plain((const char*)a.q + (src0 + u * CPR) * 16);
+    if (WITH_Q) vq[u] = ld_plain((const char*)a.q + (src0 + u * CPR) * 16);
     vk[u] = ld_stream((const char*)a.k + (src0 + u * CPR) * 16);
     vv[u] = ld_stream((const char*)a.v + (src0 + u * CPR) * 16);
   }
@@ -160,7 +162,7 @@ __global__ void __launch_bounds__(kAppendThreads)
   }
 #pragma unroll
   for (int u = 0; u < HG; ++u) {
-    st_plain((char*)a.q + (src0 + u * CPR) * 16, rotate_chunk<T>(vq[u], cs));
+    if (WITH_Q) st_plain((char*)a.q + (src0 + u * CPR) * 16, rotate_chunk<T>(vq[u], cs));
     st_plain(kpool + (dst0 + u * head_step) * 16, rotate_chunk<T>(vk[u], cs));
     st_plain(vpool + (dst0 + u * head_step) * 16, vv[u]);
   }
@@ -224,15 +226,22 @@ cudaError_t launch_rope_append(const RopeTables& rt, const Pools& pools, const A
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-#define LBM_APPEND_LAUNCH(T, C)                                                           \
-  if (hg == 4) return cudaLaunchKernelEx(&cfg, rope_append_kernel<T, C, 4>, rt, pools, a); \
-  if (hg == 2) return cudaLaunchKernelEx(&cfg, rope_append_kernel<T, C, 2>, rt, pools, a); \
-  return cudaLaunchKernelEx(&cfg, rope_append_kernel<T, C, 1>, rt, pools, a);
+#define LBM_APPEND_LAUNCH_Q(T, C, Q)                                                        \
+  if (hg == 4) return cudaLaunchKernelEx(&cfg, rope_append_kernel<T, C, 4, Q>, rt, pools, a); \
+  if (hg == 2) return cudaLaunchKernelEx(&cfg, rope_append_kernel<T, C, 2, Q>, rt, pools, a); \
+  return cudaLaunchKernelEx(&cfg, rope_append_kernel<T, C, 1, Q>, rt, pools, a);
+#define LBM_APPEND_LAUNCH(T, C)             \
+  if (a.q != nullptr) {                     \
+    LBM_APPEND_LAUNCH_Q(T, C, true)         \
+  } else {                                  \
+    LBM_APPEND_LAUNCH_Q(T, C, false)        \
+  }
   if (a.dtype == LBM_BF16 && cpr == 8) { LBM_APPEND_LAUNCH(__nv_bfloat16, 8) }
   if (a.dtype == LBM_BF16 && cpr == 16) { LBM_APPEND_LAUNCH(__nv_bfloat16, 16) }
   if (a.dtype == LBM_F32 && cpr == 16) { LBM_APPEND_LAUNCH(float, 16) }
   if (a.dtype == LBM_F32 && cpr == 32) { LBM_APPEND_LAUNCH(float, 32) }
 #undef LBM_APPEND_LAUNCH
+#undef LBM_APPEND_LAUNCH_Q
   return cudaErrorInvalidValue;
 }
 

@@ -96,11 +96,14 @@ def regen_source(cfg: workloads.StreamConfig, frame_ids: list):
 def run_stream(cfg: workloads.StreamConfig, check_frames=None, rows=None, frame_ids=None,
                tamper=None, check_pools=True, regenerate=False, report=None, decide_after=False,
                split=None, ntk_factor: float = 1.0, reset_at=(),
-               rope2d_frequency: float | None = None):
+               rope2d_frequency: float | None = None, fold_q: bool | None = None):
     """Streams every frame of cfg through the cache; checks the frames in check_frames.
 
     split, ntk_factor: RoPE variant (explicit (t, h, w) split, NTK factor), for both sides.
     rope2d_frequency: rotate with the 2D (y, x) variant of that base frequency instead.
+    fold_q: append with q = None, so the attention kernel rotates q as it loads it (it also
+    writes the rotated q it used, which is checked like the in-place rotation; bf16 only).
+    Default False: the append rotates q in place, as bench.py streams.
     reset_at: stream positions before which cache and oracle are reset (windowed streaming;
     frame_ids may then start again).
     decide_after: append every frame undecided and keep / drop it after its attention
@@ -120,6 +123,7 @@ def run_stream(cfg: workloads.StreamConfig, check_frames=None, rows=None, frame_
                               kv_source=regen_source(cfg, frame_ids) if regenerate else None,
                               split=split, ntk_factor=ntk_factor,
                               rope2d_frequency=rope2d_frequency)
+    fold_q = bool(fold_q)
     summary = []
     T = cfg.tokens
     keys = cfg.keyframes
@@ -132,8 +136,9 @@ def run_stream(cfg: workloads.StreamConfig, check_frames=None, rows=None, frame_
             q, k, v = tamper(n, q, k, v)
         qd, kd, vd = dev(q, cfg.dtype), dev(k, cfg.dtype), dev(v, cfg.dtype)
         out = torch.empty_like(qd)
-        cache.append_frame(qd, kd, vd, fid, None if decide_after else keys[n])
-        cache.attend_frame(qd, out)
+        q_rot = torch.empty_like(qd) if fold_q else None
+        cache.append_frame(None if fold_q else qd, kd, vd, fid, None if decide_after else keys[n])
+        cache.attend_frame(qd, out, q_rot_out=q_rot)
         if decide_after:
             st = cache.state()
             assert st["pending"] and st["pending_is_keyframe"] is None, fid
@@ -147,7 +152,12 @@ def run_stream(cfg: workloads.StreamConfig, check_frames=None, rows=None, frame_
         for key in ("scale_pages", "scale_frames", "window_pages", "window_frames", "free",
                     "n_special"):
             assert st[key] == r.state[key], (fid, key, st[key], r.state[key])
-        q_err = check_rope(host(qd), r.q_rot, cfg.dtype, f"frame {fid} q")
+        if fold_q:
+            # the raw q is left as it was; the rotated q is what the attention kernel used
+            np.testing.assert_array_equal(host(qd), q)
+            q_err = check_rope(host(q_rot), r.q_rot, cfg.dtype, f"frame {fid} q (in attention)")
+        else:
+            q_err = check_rope(host(qd), r.q_rot, cfg.dtype, f"frame {fid} q")
         o = host(out)[r.rows]
         rel, mx = check_attn(o, r.out, f"frame {fid} attention")
         item = {"frame": fid, "q_err": q_err, "attn_rel_l2": rel, "attn_max_abs": mx}

@@ -208,6 +208,7 @@ def test_create_argument_checks_without_gpu(lib):
     assert lib.lbm_cache_reset(None) == _lib.LBM_ERR_INVALID
     assert lib.lbm_cache_check(None) == _lib.LBM_ERR_INVALID
     assert lib.lbm_commit_frame(None, 1) == _lib.LBM_ERR_INVALID
+    assert lib.lbm_cache_set_wait_limit(None, 1000) == _lib.LBM_ERR_INVALID
     # multi-block caches: block count checked first; block calls on a null cache
     for nb in (0, -1, 1025):
         assert lib.lbm_cache_create_blocks(nb, 2, 64, 16, 6, 1, 3, 8, _lib.LBM_BF16, None,

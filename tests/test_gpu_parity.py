@@ -92,8 +92,9 @@ def test_rope2d_tables_match_oracle(head_dim, ppf, pph, ppw):
 def test_rope2d_stream_all_frames_all_rows(head_dim):
     """Fused rotate + append and attention with the 2D variant: q, pages, page table and
     outputs match the oracle rotating by (y, x) with base frequency 100."""
-    run_stream(custom_config(222 + head_dim // 64, 2, head_dim, "bf16", 7, 9, 8, 2, 1, 2),
-               rope2d_frequency=100.0)
+    cfg = custom_config(222 + head_dim // 64, 2, head_dim, "bf16", 7, 9, 8, 2, 1, 2)
+    run_stream(cfg, rope2d_frequency=100.0)
+    run_stream(cfg, rope2d_frequency=100.0, fold_q=True)
 
 
 def test_rope2d_64x64_grid_sampled():
@@ -131,10 +132,48 @@ def test_small_streams_all_frames_all_rows(cfg):
     run_stream(cfg)
 
 
+@pytest.mark.parametrize("cfg", [c for c in SMALL if c.dtype == "bf16"], ids=lambda c: c.name)
+def test_small_streams_rotation_folded_into_attention(cfg):
+    """The folded path: the append moves k and v only, the attention kernel rotates the raw q
+    in shared memory after its TMA load; the rotated q it used is checked like the in-place
+    rotation (1/2 bf16 ulp), outputs, pages and page table like every stream."""
+    run_stream(cfg, fold_q=True)
+
+
+def test_folded_rotation_argument_checks():
+    """lbm_attend_frame_qrot only for frames whose append left q to the attention; a float32
+    cache cannot fold the rotation (its attention is the SIMT kernel)."""
+    import torch
+    rope = _lib.Rope3D(64, 4, 4, 4, 6)
+    cache = _lib.PagedKVCache(rope, 2, 64, 16, 1, 1, 4, _lib.LBM_BF16)
+    q = torch.randn(22, 2, 64, device="cuda").to(torch.bfloat16)
+    k, v, out, qr = torch.randn_like(q), torch.randn_like(q), torch.empty_like(q), torch.empty_like(q)
+    cache.append_frame(q, k, v, 0, True)                  # q rotated here
+    with pytest.raises(_lib.LbmError) as e:
+        cache.attend_frame(q, out, q_rot_out=qr)
+    assert e.value.status == _lib.LBM_ERR_INVALID
+    cache.attend_frame(q, out)
+    cache.append_frame(None, k, v, 1, True)               # q left to the attention
+    cache.attend_frame(q, out, q_rot_out=qr)
+    cache.check()
+    cache.close()
+    rope32 = _lib.Rope3D(64, 4, 4, 4, 6)
+    c32 = _lib.PagedKVCache(rope32, 2, 64, 16, 1, 1, 4, _lib.LBM_F32)
+    q32 = torch.randn(22, 2, 64, device="cuda")
+    with pytest.raises(_lib.LbmError) as e:
+        c32.append_frame(None, q32, q32, 0, True)
+    assert e.value.status == _lib.LBM_ERR_UNSUPPORTED
+    c32.close()
+    rope32.close()
+    rope.close()
+
+
 @pytest.mark.parametrize("grid", ["1", "3", "16", "148"])
 def test_forced_grid_sizes_agree(grid, monkeypatch):
     monkeypatch.setenv("LBM_ATTN_GRID", grid)
-    run_stream(custom_config(205, 2, 64, "bf16", 12, 12, 8, 1, 2, 3))
+    cfg = custom_config(205, 2, 64, "bf16", 12, 12, 8, 1, 2, 3)
+    run_stream(cfg)
+    run_stream(cfg, fold_q=True)          # the folded kernel walks the same segments
 
 
 def test_keyframes_decided_after_attention():
@@ -199,6 +238,16 @@ def test_full_size_config_sampled(cid, frames):
                                                 replace=False)]))
     assert len(rows) == 128 + 7
     run_stream(cfg, check_frames=frames, rows=rows, regenerate=True)
+
+
+def test_full_size_768_folded_sampled():
+    """The folded rotation at full size (768-patch stream, frames around the window fill)."""
+    cfg = CONFIGS[1]
+    rng = np.random.default_rng(11)
+    rows = np.unique(np.concatenate([np.arange(6), [cfg.tokens - 1],
+                                     rng.choice(np.arange(6, cfg.tokens - 1), 128,
+                                                replace=False)]))
+    run_stream(cfg, check_frames=[0, 24, 25, 63], rows=rows, regenerate=True, fold_q=True)
 
 
 @pytest.mark.slow
@@ -390,6 +439,51 @@ def test_multi_block_sequence_errors():
     cache.append_frame(q, k, v, 0, True)                  # the next block in order: block 1
     cache.attend_frame(q, out)
     assert not cache.state()["pending"] and cache.state()["scale_frames"] == [0]
+    cache.check()
+    cache.close()
+    rope.close()
+
+
+@pytest.mark.parametrize("head_dim,fold", [(64, False), (64, True), (128, False), (128, True)])
+def test_wait_that_runs_out_is_reported_and_the_cache_recovers(head_dim, fold):
+    """Failure detection without a fault: with a wait limit of 1 ns the attention kernel's first
+    wait that is not already satisfied runs out; every role leaves the kernel (copies and
+    tensor-core operations already issued are drained under the full bound before tensor
+    memory is freed), lbm_cache_check reports LBM_ERR_TIMEOUT once and clears it.  With the
+    default limit restored and the cache reset, the same cache then streams frames that match
+    the oracle, so the context stays usable."""
+    import torch
+    from oracle import stream as ostream
+    from rope_paged_kv_02_b200.workloads import frame_qkv
+    from stream_check import check_attn, dev, host
+    cfg = custom_config(226 + head_dim // 64, 2, head_dim, "bf16", 10, 13, 4, 1, 1, 2)
+    rope = _lib.Rope3D(head_dim, cfg.n_frames, cfg.pph, cfg.ppw, 6)
+    cache = _lib.PagedKVCache(rope, 2, head_dim, cfg.patches, 1, 2, cfg.n_frames, _lib.LBM_BF16)
+    q, k, v = frame_qkv(cfg, 0)
+    qd, kd, vd = dev(q, "bf16"), dev(k, "bf16"), dev(v, "bf16")
+    out = torch.empty_like(qd)
+    cache.set_wait_limit(1)
+    cache.append_frame(None if fold else qd, kd, vd, 0, True)
+    cache.attend_frame(qd, out)
+    with pytest.raises(_lib.LbmError) as e:
+        cache.check()
+    assert e.value.status == _lib.LBM_ERR_TIMEOUT
+    cache.check()                                         # reported once, then cleared
+    with pytest.raises(_lib.LbmError) as e:
+        cache.set_wait_limit(3_000_000_000)               # above the 2 s default
+    assert e.value.status == _lib.LBM_ERR_INVALID
+    cache.set_wait_limit(0)
+    cache.reset()
+    so = ostream.StreamOracle(2, head_dim, cfg.pph, cfg.ppw, 1, 2, cfg.n_frames)
+    for f in range(cfg.n_frames):
+        q, k, v = frame_qkv(cfg, f)
+        qd, kd, vd = dev(q, "bf16"), dev(k, "bf16"), dev(v, "bf16")
+        out = torch.empty_like(qd)
+        cache.append_frame(None if fold else qd, kd, vd, f, True)
+        cache.attend_frame(qd, out)
+        r = so.step(f, True, q, k, v)
+        torch.cuda.synchronize()
+        check_attn(host(out), r.out, f"frame {f} after the timeout")
     cache.check()
     cache.close()
     rope.close()
