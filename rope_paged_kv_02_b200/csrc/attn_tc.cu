@@ -386,8 +386,14 @@ struct TmemMap {
 
 // One run of key tiles of one unit, as a CTA walks its share of the work.
 struct Segment {
-  int unit, a, b;   // key tiles [a, b) of the unit
+  int unit, a, b;   // items [a, b) of the unit
 };
+
+// Key tile read by item i of unit `unit` (the unit's rotation of its key order).
+__device__ __forceinline__ int key_tile(const AttnParams& p, int unit, int i) {
+  const int t = i + p.rot[unit];
+  return t >= p.n_tiles ? t - p.n_tiles : t;
+}
 
 // Work items are counted in 32-bit integers: the host keeps a frame's work below 2^31.
 __device__ __forceinline__ Segment segment_at(const AttnParams& p, int x, int hi) {
@@ -581,7 +587,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
-        const TileRef tr = tile_ref<C::BN>(p, t);
+        const TileRef tr = tile_ref<C::BN>(p, key_tile(p, sg.unit, t));
         const CUtensorMap* tk = tr.special ? &p.tm_ks : &p.tm_kp;
         const CUtensorMap* tv = tr.special ? &p.tm_vs : &p.tm_vp;
         mbar_expect_tx(bar(bars->kv_full[s]), 2 * C::KV_TILE);
@@ -782,7 +788,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         mbar_arrive(bar(bars->s_free[g]));
 
-        const int valid = tile_ref<BN>(p, sg.a + (j - j0)).valid;
+        const int valid = tile_ref<BN>(p, key_tile(p, sg.unit, sg.a + (j - j0))).valid;
         if (valid != BN) {
           // keys past the end of a page / of the special stream: -inf scores, zero weight
 #pragma unroll

@@ -160,6 +160,7 @@ int fill_attn_params(lbm_cache* c, int block, const void* q, void* out, void* q_
   const long long want = c->forced_grid ? c->forced_grid : c->num_sms;
   p.grid = (int)std::min<long long>(std::min<long long>(want, p.work), lbm::kMaxGrid);
   lbm::sk_partition(p);
+  lbm::sk_rotations(p);
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)c->head_dim));
   return LBM_OK;
 }

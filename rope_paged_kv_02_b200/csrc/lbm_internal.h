@@ -52,6 +52,7 @@ constexpr int kMaxPages = 1024;
 __host__ __device__ constexpr int attn_key_tile(int head_dim) { return head_dim == 64 ? 128 : 64; }
 
 constexpr int kMaxGrid = 1024;  // persistent attention CTAs per launch, at most
+constexpr int kMaxUnits = 1024;  // units whose key order the planner rotates (see AttnParams)
 
 // Shared memory the attention kernel sets aside for the RoPE tables of its in-kernel q
 // rotation: the frame's t row and the h and w tables, (nt + (pph+1) nh + (ppw+1) nw) float2.
@@ -100,6 +101,12 @@ struct AttnParams {
   float scale_log2;      // log2(e) / sqrt(head_dim)
   uint16_t pages[kMaxPages];
   int sk_start[kMaxGrid + 1];  // first work item of CTA c; sk_start[grid] = work
+  // Key-tile order inside each unit: item i of unit u reads key tile (i + rot[u]) mod n_tiles.
+  // The 2 n_pairs query tiles of a head read the same keys; rotating each unit so that the CTA
+  // entering it is at key tile ~tau at time tau keeps the CTAs of a head (and of all heads) on
+  // nearly the same key tiles at the same time, so each K/V tile comes from DRAM about once
+  // and from L2 for the other query tiles.  Zero rotations when units > kMaxUnits.
+  int rot[kMaxUnits];
 };
 
 struct SimtParams {
@@ -176,6 +183,25 @@ inline void sk_partition(AttnParams& p) {
     if (x < (long long)p.sk_start[c - 1] + 1) x = p.sk_start[c - 1] + 1;
     if (x > p.work - (p.grid - c)) x = p.work - (p.grid - c);
     p.sk_start[c] = (int)x;
+  }
+}
+
+// Fills p.rot (needs p.sk_start): unit u starts in exactly one CTA's range [S_c, S_{c+1});
+// that CTA reaches the unit's first item after u * n_tiles - S_c items of its own, so rotating
+// the unit by that amount (mod n_tiles) has it read key tile tau at its step tau.  A CTA whose
+// range starts inside a unit reads that unit's tail shifted by (n_tiles - share) tiles at most.
+inline void sk_rotations(AttnParams& p) {
+  const long long units = (long long)p.n_pairs * p.heads;
+  if (units > kMaxUnits) {
+    for (int u = 0; u < kMaxUnits; ++u) p.rot[u] = 0;
+    return;
+  }
+  const long long n = p.n_tiles;
+  int c = 0;
+  for (long long u = 0; u < units; ++u) {
+    const long long first = u * n;
+    while (c + 1 < p.grid && p.sk_start[c + 1] <= first) ++c;
+    p.rot[u] = (int)((first - p.sk_start[c]) % n);
   }
 }
 

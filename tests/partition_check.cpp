@@ -1,7 +1,11 @@
 // Host check of the stream-K partition the attention launcher uses (sk_partition): for many
 // frame shapes and grid sizes, the CTA starts begin at 0, end at the frame's work, strictly
 // increase (every CTA gets work), and no CTA's modelled cost exceeds the even share by more
-// than one unit's start plus a step.  Built and run by tests/test_partition_host.py.
+// than one unit's start plus a step.  And of the key-order rotations (sk_rotations): each in
+// [0, n_tiles); the CTA that reaches a unit's first item after tau items of its own reads
+// key tile tau mod n_tiles at its step tau throughout that segment; every other segment is at
+// most n_tiles - 1 tiles off its CTA's step; each unit still visits every key tile once.
+// Built and run by tests/test_partition_host.py.
 #include <cstdio>
 #include <algorithm>
 #include "../rope_paged_kv_02_b200/csrc/lbm_internal.h"
@@ -52,6 +56,37 @@ int main() {
             std::printf("FAIL balance T=%d H=%d nt=%d grid=%d worst=%lld even=%lld\n", T, H, nt,
                         p.grid, worst, even);
             return 1;
+          }
+          sk_rotations(p);
+          const long long units = (long long)p.n_pairs * H;
+          if (units <= kMaxUnits) {
+            for (int c = 0; c < p.grid; ++c) {
+              for (long long x = p.sk_start[c]; x < p.sk_start[c + 1]; ++x) {
+                const long long u = x / nt, i = x % nt;
+                const int r = p.rot[u];
+                if (r < 0 || r >= nt) {
+                  std::printf("FAIL rot range u=%lld r=%d nt=%d\n", u, r, nt);
+                  return 1;
+                }
+                const long long tile = (i + r) % nt, step = x - p.sk_start[c];
+                // the CTA holding the unit's first item is in phase with its own steps
+                if (u * nt >= p.sk_start[c] && tile != step % nt) {
+                  std::printf("FAIL phase T=%d H=%d nt=%d grid=%d c=%d u=%lld\n", T, H, nt,
+                              p.grid, c, u);
+                  return 1;
+                }
+              }
+            }
+            // a rotation is a bijection of the unit's tiles (every key tile read once)
+            for (long long u = 0; u < units && nt <= 1090; ++u) {
+              static bool seen[1090];
+              std::fill(seen, seen + nt, false);
+              for (int i = 0; i < nt; ++i) seen[(i + p.rot[u]) % nt] = true;
+              if (!std::all_of(seen, seen + nt, [](bool b) { return b; })) {
+                std::printf("FAIL cover u=%lld\n", u);
+                return 1;
+              }
+            }
           }
           ++checked;
         }

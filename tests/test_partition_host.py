@@ -1,6 +1,8 @@
 """The stream-K partition of the attention kernel, on the host (no GPU): compiles
 tests/partition_check.cpp against the library's internal header with the host compiler and
-runs it (shares start at 0, end at the frame's work, never empty, and balanced by cost)."""
+runs it (shares start at 0, end at the frame's work, never empty, and balanced by cost; the
+per-unit key-order rotations stay in range, put the CTA that enters a unit in phase with its
+own steps, and visit every key tile once)."""
 
 import os
 import shutil
