@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 #include <vector>
 
@@ -186,10 +187,12 @@ inline void sk_partition(AttnParams& p) {
   }
 }
 
-// Fills p.rot (needs p.sk_start): unit u starts in exactly one CTA's range [S_c, S_{c+1});
+// Fills p.rot (needs p.sk_start).  Unit u starts in exactly one CTA's range [S_c, S_{c+1});
 // that CTA reaches the unit's first item after u * n_tiles - S_c items of its own, so rotating
-// the unit by that amount (mod n_tiles) has it read key tile tau at its step tau.  A CTA whose
-// range starts inside a unit reads that unit's tail shifted by (n_tiles - share) tiles at most.
+// the unit by that amount (mod n_tiles) has it read key tile tau at its step tau.  When the
+// next CTA holds a longer part of the unit (from item a = S_{c+1} - u * n_tiles, at its step
+// 0), the unit is rotated for that CTA instead (by -a), so the larger part of every unit is
+// read in phase; the other part is off by less than n_tiles.
 inline void sk_rotations(AttnParams& p) {
   const long long units = (long long)p.n_pairs * p.heads;
   if (units > kMaxUnits) {
@@ -199,9 +202,16 @@ inline void sk_rotations(AttnParams& p) {
   const long long n = p.n_tiles;
   int c = 0;
   for (long long u = 0; u < units; ++u) {
-    const long long first = u * n;
+    const long long first = u * n, end = first + n;
     while (c + 1 < p.grid && p.sk_start[c + 1] <= first) ++c;
-    p.rot[u] = (int)((first - p.sk_start[c]) % n);
+    const long long own = std::min<long long>(p.sk_start[c + 1], end) - first;
+    const long long next = c + 1 < p.grid ? std::min<long long>(p.sk_start[c + 2], end) -
+                                                std::min<long long>(p.sk_start[c + 1], end)
+                                          : 0;
+    if (next > own)
+      p.rot[u] = (int)((n - (p.sk_start[c + 1] - first) % n) % n);
+    else
+      p.rot[u] = (int)((first - p.sk_start[c]) % n);
   }
 }
 

@@ -2,9 +2,9 @@
 // frame shapes and grid sizes, the CTA starts begin at 0, end at the frame's work, strictly
 // increase (every CTA gets work), and no CTA's modelled cost exceeds the even share by more
 // than one unit's start plus a step.  And of the key-order rotations (sk_rotations): each in
-// [0, n_tiles); the CTA that reaches a unit's first item after tau items of its own reads
-// key tile tau mod n_tiles at its step tau throughout that segment; every other segment is at
-// most n_tiles - 1 tiles off its CTA's step; each unit still visits every key tile once.
+// [0, n_tiles); the CTA holding the larger part of a unit (of the first two CTAs on it) reads
+// key tile tau mod n_tiles at its step tau throughout that part; each unit still visits every
+// key tile once.
 // Built and run by tests/test_partition_host.py.
 #include <cstdio>
 #include <algorithm>
@@ -69,8 +69,18 @@ int main() {
                   return 1;
                 }
                 const long long tile = (i + r) % nt, step = x - p.sk_start[c];
-                // the CTA holding the unit's first item is in phase with its own steps
-                if (u * nt >= p.sk_start[c] && tile != step % nt) {
+                // the CTA holding the larger part of the unit (of the first two) reads it in
+                // phase with its own steps
+                const long long first = u * nt, end = first + nt;
+                int c0 = 0;
+                while (c0 + 1 < p.grid && p.sk_start[c0 + 1] <= first) ++c0;
+                const long long own = std::min<long long>(p.sk_start[c0 + 1], end) - first;
+                const long long next =
+                    c0 + 1 < p.grid ? std::min<long long>(p.sk_start[c0 + 2], end) -
+                                          std::min<long long>(p.sk_start[c0 + 1], end)
+                                    : 0;
+                const int phased = next > own ? c0 + 1 : c0;
+                if (c == phased && tile != step % nt) {
                   std::printf("FAIL phase T=%d H=%d nt=%d grid=%d c=%d u=%lld\n", T, H, nt,
                               p.grid, c, u);
                   return 1;
