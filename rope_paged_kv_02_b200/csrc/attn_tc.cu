@@ -324,6 +324,16 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   return d;
 }
 
+// The eight floats of four packed pairs, summed pairwise.
+__device__ __forceinline__ float sum_f2x4(const uint64_t* v) {
+  float a0, a1, b0, b1, c0, c1, d0, d1;
+  unpack_f2(v[0], a0, a1);
+  unpack_f2(v[1], b0, b1);
+  unpack_f2(v[2], c0, c1);
+  unpack_f2(v[3], d0, d1);
+  return ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
+}
+
 // Key tile t of the visible list: pool (patch or special), first pool row, valid keys.
 struct TileRef {
   bool special;
@@ -331,12 +341,23 @@ struct TileRef {
   int valid;
 };
 
+// Page index of patch tile t, t / tiles_per_page: a multiply-high with the host's
+// tpp_magic = ceil(2^32 / tiles_per_page), exact while t * tiles_per_page < 2^32 (the host
+// sets tpp_magic = 0 for frames where that could fail, and then this divides).
+__device__ __forceinline__ int tile_page(const AttnParams& p, int t) {
+  if (p.tiles_per_page == 1) return t;
+  return p.tpp_magic ? (int)__umulhi((uint32_t)t, p.tpp_magic) : t / p.tiles_per_page;
+}
+__device__ __forceinline__ int tile_in_page(const AttnParams& p, int t) {
+  return t - tile_page(p, t) * p.tiles_per_page;
+}
+
 template <int BN>
 __device__ __forceinline__ TileRef tile_ref(const AttnParams& p, int t) {
   const int npt = p.n_pages * p.tiles_per_page;
   TileRef r;
   if (t < npt) {
-    const int pi = t / p.tiles_per_page;
+    const int pi = tile_page(p, t);
     const int i = t - pi * p.tiles_per_page;
     r.special = false;
     r.row0 = (int)p.pages[pi] * p.page_stride + BN * i;
@@ -348,6 +369,15 @@ __device__ __forceinline__ TileRef tile_ref(const AttnParams& p, int t) {
     r.valid = min(BN, p.n_special - BN * i);
   }
   return r;
+}
+
+// Valid keys of key tile t (see tile_ref), without a division when every patch tile is full.
+template <int BN>
+__device__ __forceinline__ int tile_valid(const AttnParams& p, int t) {
+  const int npt = p.n_pages * p.tiles_per_page;
+  if (t >= npt) return min(BN, p.n_special - BN * (t - npt));
+  if (p.patches % BN == 0) return BN;
+  return min(BN, p.patches - BN * tile_in_page(p, t));
 }
 
 struct Bars {
@@ -775,8 +805,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int sb = TM::buf(j);
         const uint32_t tS = lane_base + TM::S(sb);
         const uint32_t tP = lane_base + TM::P(sb);
-        if (!__all_sync(kFull, mbar_wait(bar(bars->s_full[g][sb]), TM::par(j), wa, 
-                                         6))) {
+        // keys of this tile: at head_dim 128 computed before the wait, off the score -> max
+        // chain; at head_dim 64 (every register taken) after the scores are in
+        int valid = D == 128 ? tile_valid<BN>(p, key_tile(p, sg.unit, sg.a + (j - j0))) : BN;
+        if (!__all_sync(kFull, mbar_wait(bar(bars->s_full[g][sb]), TM::par(j), wa, 6))) {
           ok = false;
           break;
         }
@@ -785,10 +817,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < BN / 32; ++c) tmem_ld32(tS + 32 * c, S + 32 * c);
         tmem_wait_ld();
         reg_fence<BN>(S);
-        tc_fence_before();
-        mbar_arrive(bar(bars->s_free[g]));
+        if (TM::NB == 1) {
+          // one S buffer: the next Q.K^T may overwrite it once every thread has read it
+          tc_fence_before();
+          mbar_arrive(bar(bars->s_free[g]));
+        }
 
-        const int valid = tile_ref<BN>(p, key_tile(p, sg.unit, sg.a + (j - j0))).valid;
+        if (D == 64) valid = tile_valid<BN>(p, key_tile(p, sg.unit, sg.a + (j - j0)));
         if (valid != BN) {
           // keys past the end of a page / of the special stream: -inf scores, zero weight
 #pragma unroll
@@ -843,14 +878,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tmem_st16(tP + 16 * c, pk);
         }
-        {
-          float a0, a1, b0, b1, c0, c1, d0, d1;
-          unpack_f2(l4[0], a0, a1);
-          unpack_f2(l4[1], b0, b1);
-          unpack_f2(l4[2], c0, c1);
-          unpack_f2(l4[3], d0, d1);
-          l += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
-        }
+        l += sum_f2x4(l4);
         if (__any_sync(kFull, rescale) && j > j0) {
           // O holds sum_{i<j} P_i V_i relative to the old max: scale it before PV_j lands
           if (TM::NB == 2 &&

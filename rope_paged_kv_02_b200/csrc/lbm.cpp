@@ -151,9 +151,11 @@ int fill_attn_params(lbm_cache* c, int block, const void* q, void* out, void* q_
   p.page_stride = bk.pools.page_stride;
   const int kt = lbm::attn_key_tile(c->head_dim);  // keys per attention key tile
   p.tiles_per_page = (c->patches + kt - 1) / kt;
+  p.tpp_magic = 0u;  // set below once n_tiles is known
   p.n_pages = n_pages;
   p.n_special = n_sp;
   p.n_tiles = p.n_pages * p.tiles_per_page + (n_sp + kt - 1) / kt;
+  p.tpp_magic = lbm::tile_div_magic(p.tiles_per_page, p.n_tiles);
   p.n_pairs = ((T + 127) / 128 + 1) / 2;
   p.work = (long long)p.n_pairs * c->heads * p.n_tiles;
   if (p.work >= (1LL << 31)) return LBM_ERR_UNSUPPORTED;  // the kernel counts in 32 bits

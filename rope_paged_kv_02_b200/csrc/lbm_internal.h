@@ -93,6 +93,7 @@ struct AttnParams {
   int patches;           // valid tokens per patch page
   int page_stride;
   int tiles_per_page;    // key tiles per patch page: ceil(patches / attn_key_tile(D))
+  uint32_t tpp_magic;    // ceil(2^32 / tiles_per_page) (tiles_per_page > 1): division by it
   int n_pages;           // visible patch pages
   int n_special;         // visible special tokens
   int n_tiles;           // n_pages * tiles_per_page + ceil(n_special / attn_key_tile(D))
@@ -213,6 +214,14 @@ inline void sk_rotations(AttnParams& p) {
     else
       p.rot[u] = (int)((first - p.sk_start[c]) % n);
   }
+}
+
+// Multiplier m = ceil(2^32 / d) with which floor(t * m / 2^32) = t / d for every t < n
+// (exact while n * d <= 2^32: the error t * (m - 2^32/d) / 2^32 stays below 1/d); 0 when that
+// does not hold or d == 1, and the kernel then divides.
+inline uint32_t tile_div_magic(int d, long long n) {
+  if (d <= 1 || (unsigned long long)n * (unsigned long long)d > (1ull << 32)) return 0u;
+  return (uint32_t)(((1ull << 32) + (unsigned long long)d - 1) / (unsigned long long)d);
 }
 
 // true when some unit is shared by two CTAs (then the combine kernel must run)

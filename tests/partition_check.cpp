@@ -4,7 +4,8 @@
 // than one unit's start plus a step.  And of the key-order rotations (sk_rotations): each in
 // [0, n_tiles); the CTA holding the larger part of a unit (of the first two CTAs on it) reads
 // key tile tau mod n_tiles at its step tau throughout that part; each unit still visits every
-// key tile once.
+// key tile once.  And the multiply-high division of tile indices (tile_div_magic): exact for
+// every index below the tile count it is enabled for, off where it could fail.
 // Built and run by tests/test_partition_host.py.
 #include <cstdio>
 #include <algorithm>
@@ -100,6 +101,33 @@ int main() {
           }
           ++checked;
         }
+  // the multiply-high division of tile indices by tiles per page (tile_div_magic)
+  for (int d : {2, 3, 5, 6, 7, 8, 9, 17, 63, 64, 65, 127, 1000, 2047, 4095, 16384, 65535}) {
+    for (long long n : {100LL, 70000LL, 1LL << 17, 1LL << 20, 1LL << 24}) {
+      const uint32_t m = tile_div_magic(d, n);
+      if ((unsigned long long)n * d > (1ull << 32)) {
+        if (m != 0) {
+          std::printf("FAIL magic should be off d=%d n=%lld\n", d, n);
+          return 1;
+        }
+        continue;
+      }
+      const long long step = n > (1LL << 20) ? 7 : 1;
+      for (long long t = 0; t < n; t += step) {
+        const long long q = (long long)(((unsigned long long)t * m) >> 32);
+        if (q != t / d) {
+          std::printf("FAIL magic d=%d t=%lld\n", d, t);
+          return 1;
+        }
+      }
+      for (long long t = n - 1; t >= 0 && t > n - 4096; --t) {   // the largest indices
+        if ((long long)(((unsigned long long)t * m) >> 32) != t / d) {
+          std::printf("FAIL magic top d=%d t=%lld\n", d, t);
+          return 1;
+        }
+      }
+    }
+  }
   std::printf("ok %lld\n", checked);
   return 0;
 }
