@@ -197,14 +197,14 @@ def test_non_contiguous_frame_indices():
     run_stream(cfg, frame_ids=[0, 3, 4, 10, 11, 20, 57, 58])
 
 
-def _needle(cfg, n_needle_frame, target_frame, row, boost):
-    """Tamper hook: plant at frame n_needle_frame a key equal to boost * (rotated q of
-    target_frame, row), and scale every q by 4 (peaked softmax: scores of std 4, the
-    needle's about 25)."""
+def _needle(cfg, n_needle_frame, target_frame, row, boost, page_pos=5):
+    """Tamper hook: plant at frame n_needle_frame, page position page_pos, a key equal to
+    boost * (rotated q of target_frame, row), and scale every q by 4 (peaked softmax: scores
+    of std 4, the needle's about 25)."""
     from rope_paged_kv_02_b200.workloads import frame_qkv, round_bf16
     q_t, _, _ = frame_qkv(cfg, target_frame)
     q_rot = rope3d.rotate_frame(q_t.astype(np.float64) * 4.0, target_frame, 6, cfg.pph, cfg.ppw)
-    slot = 6 + 5
+    slot = 6 + page_pos
     pos = rope3d.token_positions(n_needle_frame, 6, cfg.pph, cfg.ppw)[slot:slot + 1]
     kneedle = rope3d.rotate(boost * q_rot[row:row + 1],
                             -rope3d.angles_for_positions(pos, cfg.head_dim))[0]
@@ -222,6 +222,17 @@ def _needle(cfg, n_needle_frame, target_frame, row, boost):
 def test_peaked_softmax_with_needle_key():
     cfg = custom_config(207, 2, 64, "bf16", 10, 13, 6, 1, 1, 3)
     tamper = _needle(cfg, 2, 5, 0, 0.2)
+    run_stream(cfg, tamper=tamper)
+
+
+@pytest.mark.parametrize("page_pos", [40, 70, 100, 129])
+def test_needle_key_past_the_first_score_chunk(page_pos):
+    """head_dim 64 reads a 128-key tile in four 32-key chunks and may move its reference max
+    at any chunk: a needle at key 40, 70 or 100 of its page's first tile (chunks 1, 2, 3) or
+    at key 129 (second tile) makes the max jump after P of earlier chunks was produced, so
+    those are scaled again; the output must still match the oracle."""
+    cfg = custom_config(207, 2, 64, "bf16", 10, 13, 6, 1, 1, 3)
+    tamper = _needle(cfg, 2, 5, 0, 0.2, page_pos=page_pos)
     run_stream(cfg, tamper=tamper)
 
 
