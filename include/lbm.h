@@ -149,7 +149,9 @@ LBM_API void lbm_rope_destroy(lbm_rope_t* rope);
  *   specials_per_frame must equal rope's patch_start_idx and be 6
  *   scale_frames, sliding_window  >= 0; scale_frames + sliding_window + 1 <= LBM_MAX_PAGES
  *   max_frames         keyframes the special stream can hold (>= 1)
- *   dtype              LBM_BF16 (tensor-core path) or LBM_F32 (exact SIMT path)
+ *   dtype              LBM_BF16 (tensor-core path) or LBM_F32 (exact SIMT path); a bf16
+ *                      cache needs a compute capability 10.0 device (B200) with the
+ *                      attention kernel's shared memory, else LBM_ERR_UNSUPPORTED
  *   rope               tables built for the same head_dim / grid; must outlive the cache
  * Device memory: K and V patch pools [heads][P*stride][head_dim] with P = scale_frames +
  * sliding_window + 1 pages and stride = patches_per_frame rounded up to 128 (zero-filled);

@@ -425,6 +425,21 @@ int lbm_cache_create_blocks(int num_blocks, int heads, int head_dim, int patches
   c->rope = rope;
   cudaGetDevice(&c->device);
   cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device);
+  if (dtype == LBM_BF16) {
+    // the bf16 attention is tcgen05 code built for sm_100a: it runs on compute capability
+    // 10.0 only, with the dynamic shared memory of its larger (folded) instance
+    int major = 0, minor = 0, optin = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, c->device);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, c->device);
+    cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, c->device);
+    const size_t need = std::max(lbm::attn_tc_smem_bytes(head_dim, false),
+                                 lbm::attn_tc_smem_bytes(head_dim, true));
+    if (major != 10 || minor != 0 || (size_t)optin < need) {
+      cudaGetLastError();
+      delete c;
+      return LBM_ERR_UNSUPPORTED;
+    }
+  }
   if (const char* env = std::getenv("LBM_ATTN_GRID")) {
     const int v = std::atoi(env);
     if (v >= 1 && v <= 4 * c->num_sms && v <= lbm::kMaxGrid) c->forced_grid = v;

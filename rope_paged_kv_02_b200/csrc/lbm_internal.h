@@ -132,6 +132,7 @@ cudaError_t launch_rope_append(const RopeTables& rt, const Pools& pools,
                                const AppendArgs& a, cudaStream_t s);
 
 // attn_tc.cu (bf16, tcgen05)
+// dynamic shared memory of one attention CTA (checked against the device at cache creation)
 size_t attn_tc_smem_bytes(int head_dim, bool fold);
 cudaError_t launch_attn_tc(const AttnParams& p, int head_dim, cudaStream_t s);
 // merges the partial results of every unit that spans more than one CTA
