@@ -421,9 +421,10 @@ struct Segment {
   int unit, a, b;   // items [a, b) of the unit
 };
 
-// Key tile read by item i of unit `unit` (the unit's rotation of its key order).
+// Key tile read by item i of unit `unit` (the unit's rotation of its key order; units past
+// the rotation table, kMaxUnits, keep the natural order).
 __device__ __forceinline__ int key_tile(const AttnParams& p, int unit, int i) {
-  const int t = i + p.rot[unit];
+  const int t = i + (unit < kMaxUnits ? p.rot[unit] : 0);
   return t >= p.n_tiles ? t - p.n_tiles : t;
 }
 

@@ -107,7 +107,8 @@ struct AttnParams {
   // The 2 n_pairs query tiles of a head read the same keys; rotating each unit so that the CTA
   // entering it is at key tile ~tau at time tau keeps the CTAs of a head (and of all heads) on
   // nearly the same key tiles at the same time, so each K/V tile comes from DRAM about once
-  // and from L2 for the other query tiles.  Zero rotations when units > kMaxUnits.
+  // and from L2 for the other query tiles.  When units > kMaxUnits no unit is rotated (the
+  // kernel reads rot[u] only for u < kMaxUnits).
   int rot[kMaxUnits];
 };
 

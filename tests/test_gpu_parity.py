@@ -498,3 +498,12 @@ def test_wait_that_runs_out_is_reported_and_the_cache_recovers(head_dim, fold):
     cache.check()
     cache.close()
     rope.close()
+
+
+@pytest.mark.parametrize("head_dim", [64, 128])
+def test_more_units_than_the_rotation_table(head_dim):
+    """1100 heads of a 22-token frame: 1100 (query-tile pair, head) units, more than the
+    1024 whose key order the planner rotates, so units 1024..1099 read their keys in the
+    natural order; every head must still match the oracle."""
+    cfg = custom_config(222, 1100, head_dim, "bf16", 4, 4, 6, 1, 1, 3)
+    run_stream(cfg, check_frames=[0, 3, 5])
