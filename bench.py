@@ -50,16 +50,60 @@ UNIT = "frames/s"
 TRAFFIC_PROFILES = {4: "attn_tc_large4096.md", 1: "attn_tc_stream768.md"}
 
 
-def _peaks():
-    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(path):
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def _peak_number(d, key):
+    """The number stored under key in the peaks file: a plain number, or a record holding one
+    (value / median / mean), at the top level or inside a nested record; None if absent."""
+    def as_num(v):
+        if isinstance(v, bool):
+            return None
+        if isinstance(v, (int, float)):
+            return float(v)
+        if isinstance(v, dict):
+            for k in ("value", "median", "mean"):
+                if isinstance(v.get(k), (int, float)) and not isinstance(v.get(k), bool):
+                    return float(v[k])
+        return None
+    if not isinstance(d, dict):
+        return None
+    if key in d and as_num(d[key]) is not None:
+        return as_num(d[key])
+    for v in d.values():
+        r = _peak_number(v, key) if isinstance(v, dict) else None
+        if r is not None:
+            return r
+    return None
+
+
+def _peaks(path=None):
+    """Roofline denominators: MEASURED_PEAKS.json when it holds them, else the fallback figures
+    (a figure missing from the file falls back alone, and the source says so)."""
+    path = path or os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if not os.path.exists(path):
+        return dict(FALLBACK_PEAKS, source="fallback")
+    try:
         with open(path) as f:
             d = json.load(f)
-        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
-                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
-                "source": "measured"}
-    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
-            "source": "fallback"}
+    except (OSError, ValueError) as e:
+        return dict(FALLBACK_PEAKS, source=f"fallback (MEASURED_PEAKS.json unreadable: {e})")
+    out, missing = {}, []
+    for key in ("hbm_gbs", "bf16_tflops"):
+        v = _peak_number(d, key)
+        if v is None or v <= 0:
+            missing.append(key)
+            v = FALLBACK_PEAKS[key]
+        out[key] = v
+    sus = _peak_number(d, "bf16_tflops_sustained")
+    if sus and sus > 0:
+        out["bf16_tflops_sustained"] = sus
+    elif "bf16_tflops" in missing:
+        out["bf16_tflops_sustained"] = FALLBACK_PEAKS["bf16_tflops_sustained"]
+    else:
+        out["bf16_tflops_sustained"] = out["bf16_tflops"]
+    out["source"] = "measured" if not missing else "measured (fallback for " + ", ".join(missing) + ")"
+    return out
 
 
 def tensor_peak(peaks: dict, clocks: dict) -> tuple[float, str]:

@@ -8,6 +8,7 @@ import subprocess
 import sys
 
 import numpy as np
+import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, ROOT)
@@ -46,3 +47,30 @@ def test_frame_work_follows_retained_key_count():
             assert keys[f] == nk
             assert flops[f] == 4.0 * cfg.tokens * nk * cfg.heads * cfg.head_dim
         assert np.all(nbytes == 6.0 * cfg.tokens * cfg.heads * cfg.head_dim * 2)
+
+
+@pytest.mark.parametrize("content,expect", [
+    ('{"hbm_gbs": 7000, "bf16_tflops": 1600, "bf16_tflops_sustained": 1380}',
+     (7000.0, 1600.0, 1380.0, "measured")),
+    ('{"hbm_gbs": {"value": 7100}, "bf16_tflops": {"median": 1610}}',
+     (7100.0, 1610.0, 1610.0, "measured")),
+    ('{"gpu0": {"hbm_gbs": 7050, "bf16_tflops": 1620, "bf16_tflops_sustained": 1390}}',
+     (7050.0, 1620.0, 1390.0, "measured")),
+    ('{"hbm_gbs": 7000}', (7000.0, 1590.0, 1400.0, "measured (fallback for bf16_tflops)")),
+    ("not json", (6650.0, 1590.0, 1400.0, "fallback (MEASURED_PEAKS.json unreadable")),
+])
+def test_peaks_file_shapes(tmp_path, content, expect):
+    """The roofline denominators are read from the peaks file whatever its nesting; a figure
+    it lacks, or an unreadable file, falls back to the recipe's figures and says so."""
+    import bench
+    p = tmp_path / "MEASURED_PEAKS.json"
+    p.write_text(content)
+    got = bench._peaks(str(p))
+    assert (got["hbm_gbs"], got["bf16_tflops"], got["bf16_tflops_sustained"]) == expect[:3]
+    assert got["source"].startswith(expect[3])
+
+
+def test_peaks_fallback_without_file(tmp_path):
+    import bench
+    got = bench._peaks(str(tmp_path / "absent.json"))
+    assert got["source"] == "fallback" and got["hbm_gbs"] == 6650.0
