@@ -171,9 +171,37 @@ class ClockSampler:
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, device_index: int):
-        self.idx = device_index
+        self.idx = self.smi_id(device_index)
         self.proc = None
         self.lines = []
+
+    @staticmethod
+    def smi_id(device_index: int) -> str:
+        """nvidia-smi's name for CUDA device device_index: its UUID or PCI bus id (the CUDA
+        ordinal and nvidia-smi's index differ under CUDA_VISIBLE_DEVICES), checked by one
+        query; the ordinal itself when neither answers."""
+        cands = []
+        try:
+            import torch
+            if torch.cuda.is_available():
+                pr = torch.cuda.get_device_properties(device_index)
+                u = str(getattr(pr, "uuid", "") or "")
+                if u:
+                    cands.append(u if u.startswith("GPU-") else "GPU-" + u)
+                cands.append("%08X:%02X:%02X.0" % (pr.pci_domain_id, pr.pci_bus_id,
+                                                   pr.pci_device_id))
+        except Exception:
+            pass
+        for c in cands:
+            try:
+                r = subprocess.run(["nvidia-smi", f"--id={c}", "--query-gpu=index",
+                                    "--format=csv,noheader"], capture_output=True, text=True,
+                                   timeout=20)
+                if r.returncode == 0 and r.stdout.strip():
+                    return c
+            except (OSError, subprocess.SubprocessError):
+                break
+        return str(device_index)
 
     def __enter__(self):
         try:
@@ -216,9 +244,10 @@ class ClockSampler:
                 if v.lower() == "active":
                     reasons.add(n)
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0,
+                    "gpu": self.idx}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "gpu": self.idx}
 
 
 def dist_setup(n_gpus: int):
