@@ -421,10 +421,14 @@ struct Segment {
   int unit, a, b;   // items [a, b) of the unit
 };
 
-// Key tile read by item i of unit `unit` (the unit's rotation of its key order; units past
-// the rotation table, kMaxUnits, keep the natural order).
-__device__ __forceinline__ int key_tile(const AttnParams& p, int unit, int i) {
-  const int t = i + (unit < kMaxUnits ? p.rot[unit] : 0);
+// Rotation of unit `unit`'s key order (units past the rotation table, kMaxUnits, keep the
+// natural order).  Read once per segment: an indexed read of the parameter block.
+__device__ __forceinline__ int unit_rot(const AttnParams& p, int unit) {
+  return unit < kMaxUnits ? p.rot[unit] : 0;
+}
+// Key tile read by item i of a unit rotated by rot.
+__device__ __forceinline__ int key_tile(const AttnParams& p, int rot, int i) {
+  const int t = i + rot;
   return t >= p.n_tiles ? t - p.n_tiles : t;
 }
 
@@ -605,6 +609,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const int n_q = seg_nq(p, sg, q_tiles);
       const int head = seg_head(p, sg);
+      const int rot = unit_rot(p, sg.unit);
       mbar_expect_tx(bar(bars->q_loaded), n_q * C::Q_TILE);
       for (int g = 0; g < n_q; ++g) {
 #pragma unroll
@@ -620,7 +625,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
-        const TileRef tr = tile_ref<C::BN>(p, key_tile(p, sg.unit, t));
+        const TileRef tr = tile_ref<C::BN>(p, key_tile(p, rot, t));
         const CUtensorMap* tk = tr.special ? &p.tm_ks : &p.tm_kp;
         const CUtensorMap* tv = tr.special ? &p.tm_vs : &p.tm_vp;
         mbar_expect_tx(bar(bars->kv_full[s]), 2 * C::KV_TILE);
@@ -800,6 +805,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (g >= seg_nq(p, sg, q_tiles)) continue;
       const int n = sg.b - sg.a;
       const int j0 = jg;
+      // head_dim 128 reads the unit's rotation once per segment (the valid-key count is
+      // computed before the score wait); head_dim 64 per tile (measured faster there)
+      const int rot = D == 128 ? unit_rot(p, sg.unit) : 0;
       float m = -INFINITY;  // running max (log2 domain) the P values and O are relative to
       float l = 0.f;
       for (int j = j0; ok && j < j0 + n; ++j) {
@@ -810,7 +818,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t tP = lane_base + TM::P(sb);
         // keys of this tile: at head_dim 128 computed before the wait, off the score -> max
         // chain; at head_dim 64 (every register taken) after the scores are in
-        int valid = D == 128 ? tile_valid<BN>(p, key_tile(p, sg.unit, sg.a + (j - j0))) : BN;
+        int valid = D == 128 ? tile_valid<BN>(p, key_tile(p, rot, sg.a + (j - j0))) : BN;
         if (!__all_sync(kFull, mbar_wait(bar(bars->s_full[g][sb]), TM::par(j), wa, 6))) {
           ok = false;
           break;
@@ -826,7 +834,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(bar(bars->s_free[g]));
         }
 
-        if (D == 64) valid = tile_valid<BN>(p, key_tile(p, sg.unit, sg.a + (j - j0)));
+        if (D == 64) valid = tile_valid<BN>(p, key_tile(p, unit_rot(p, sg.unit), sg.a + (j - j0)));
         if (valid != BN) {
           // keys past the end of a page / of the special stream: -inf scores, zero weight
 #pragma unroll
