@@ -36,6 +36,8 @@
 // which drains outstanding copies / MMAs (bounded) and frees tensor memory.
 #include <cuda_bf16.h>
 
+#include <mutex>
+
 #include "../../include/lbm.h"
 #include "lbm_internal.h"
 
@@ -1116,13 +1118,23 @@ size_t attn_tc_smem_bytes(int head_dim, bool fold) {
 
 namespace {
 
+constexpr int kMaxAttnDevices = 64;
+
+// The shared-memory opt-in of a kernel is set per device: once for every device this process
+// launches the kernel on (thread-safe, no allocation).
 template <int D, bool FOLD>
 cudaError_t prepare_attn_tc() {
-  static cudaError_t state = cudaErrorNotReady;
-  if (state == cudaErrorNotReady)
-    state = cudaFuncSetAttribute(attn_tc_kernel<D, FOLD>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D, FOLD>::SMEM);
-  return state;
+  static std::once_flag once[kMaxAttnDevices];
+  static cudaError_t state[kMaxAttnDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxAttnDevices)
+    return cudaErrorInvalidDevice;
+  std::call_once(once[dev], [dev] {
+    state[dev] = cudaFuncSetAttribute(attn_tc_kernel<D, FOLD>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      Cfg<D, FOLD>::SMEM);
+  });
+  return state[dev];
 }
 
 }  // namespace
